@@ -1,0 +1,630 @@
+#!/usr/bin/env python3
+"""Benchmark of the NVFP4 KV-cache path on B200: GB/s of algorithmic bytes moved, the
+fraction of the HBM roofline, and tokens/s.
+
+Default workload (``--workload rollout``): a self-forcing video rollout on a Wan-shaped
+cache -- 30 layers x {K, V}, 12 heads, head_dim 128, 1560 tokens per frame, capacity 60
+frames. One bench step is the whole 60-frame rollout: every frame appends 1560 new
+tokens per layer through kvq_append_batch (quantize-on-write, rule mse) and then
+dequantizes every layer's K and V prefix into one reused bf16 buffer through
+kvq_dequantize_cache_batch. This one workload runs every stage of the path: cache
+sizing, per-chunk amax, block scales, e2m1 packing, and dequantization.
+
+Other workloads: ``single`` ([4096,128], static_6), ``layer`` (one layer's K and V of
+[1,24,4680,128], mse), ``cache`` (30 layers x {K,V} of [1,24,32760,128]; quantize all,
+dequantize per layer), ``sweep`` ([T,128], --tokens).
+
+Timing: each bench step is captured as CUDA graphs (one per segment: an append, a
+layer loop of reads, ...), replayed with CUDA events between segments on the launching
+stream; W warm-up steps, then K timed steps between a barrier and a device synchronize;
+the step time is the max over ranks. Workloads smaller than L2 flush it (a 256 MB
+write) between timed steps, outside the events.
+
+``--impl reference`` times the CPU oracle (the plain C restatement of the method) on a
+bounded sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 KV quant+dequant GB/s (bytes moved) and % of B200 HBM peak; tokens/s"
+B_QUANT = 2.5625   # bf16 read + 0.5 B codes + 1/16 B scale written, per element
+B_AMAX = 2.0       # bf16 read, per element
+B_DEQUANT = 2.5625  # 0.5625 B read + bf16 written, per element
+L2_BYTES = 126 * 2 ** 20
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML every 100 ms."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(device_index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, keep running
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": f"NVML unavailable: {self.err}"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------- workloads
+
+class Segment:
+    """A unit of GPU work captured as one CUDA graph; `kind` groups segments for the
+    per-kernel timing, `launches` counts the library's kernels it runs."""
+
+    def __init__(self, kind, fn, launches, bytes_alg, h2d=None):
+        self.kind, self.fn, self.launches, self.bytes_alg, self.h2d = kind, fn, launches, bytes_alg, h2d
+        self.graph = None
+
+
+class Rollout:
+    name = "rollout"
+
+    def __init__(self, args, rank):
+        self.layers, self.heads, self.tokens, self.frames, self.D = 30, 12, 1560, 60, 128
+        if args.small:
+            self.layers, self.heads, self.tokens, self.frames = 2, 2, 120, 6
+        self.rule = args.rule or "mse"
+        self.rank = rank
+        self.rpc = self.tokens * self.heads
+        self.chunk_elems = self.rpc * self.D
+        self.config = {
+            "workload": f"rollout append+dequant: {self.layers} layers x {{K,V}}, {self.heads} heads, "
+                        f"{self.tokens} tokens/frame x {self.frames} frames, head_dim {self.D}, Student-t(4), "
+                        f"rule {self.rule}",
+            "model": "Wan-shaped self-forcing KV cache (synthetic)",
+            "global_batch": 1, "seq_len": self.tokens * self.frames, "parallelism": "replica per GPU",
+            "l2": "inputs larger than L2 (per-step appends and the growing cache exceed 126 MB)",
+        }
+
+    def setup(self, kvq, inputs, dev):
+        T = 2 * self.layers
+        self.caches = kvq.allocate_caches(self.layers, self.heads, self.frames * self.tokens, self.D, self.tokens, dev)
+        self.sizes = kvq.kvq_cache_bytes(self.layers, self.heads, self.frames * self.tokens, self.D, self.tokens)
+        self.x = torch.empty((self.frames, T, self.chunk_elems), dtype=torch.bfloat16, device=dev)
+        for f in range(self.frames):
+            for t in range(T):
+                self.x[f, t] = inputs.rollout_chunk(f + self.frames * self.rank, t, heads=self.heads,
+                                                    tokens=self.tokens, device=dev).reshape(-1)
+        cap = self.frames * self.chunk_elems
+        self.yk = torch.empty(cap, dtype=torch.bfloat16, device=dev)
+        self.yv = torch.empty(cap, dtype=torch.bfloat16, device=dev)
+        self.kvq = kvq
+
+    def segments(self):
+        kvq, T, segs = self.kvq, 2 * self.layers, []
+        for f in range(self.frames):
+            xs = [self.x[f, t] for t in range(T)]
+
+            def app(f=f, xs=xs):
+                kvq.kvq_append_batch(self.caches, [f * self.rpc] * T, xs, self.rule)
+            segs.append(Segment("append", app, 3 * math.ceil(T / kvq.MAX_BATCH),
+                                T * self.chunk_elems * (B_AMAX + B_QUANT), h2d=(self.x[f],)))
+            rows = (f + 1) * self.rpc
+
+            def deq(rows=rows):
+                for l in range(self.layers):
+                    kvq.kvq_dequantize_cache_batch(self.caches[2 * l:2 * l + 2], 0, rows,
+                                                   [self.yk[:rows * self.D], self.yv[:rows * self.D]])
+            segs.append(Segment("dequant", deq, self.layers, T * rows * self.D * B_DEQUANT))
+        return segs
+
+    def d2h(self):
+        c0 = self.caches[0]
+        # the three backing buffers of every cache (allocate_caches carves them contiguously)
+        return [c0.packed._base if c0.packed._base is not None else c0.packed,
+                c0.scales._base if c0.scales._base is not None else c0.scales,
+                c0.amax._base if c0.amax._base is not None else c0.amax]
+
+    def tokens_per_step(self):
+        return self.tokens * self.frames
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        """Layer 0's K and V through the rollout until the time budget is spent."""
+        caches = [orc.Cache(self.frames * self.rpc, self.rpc, self.D) for _ in range(2)]
+        spent, nbytes, f = 0.0, 0.0, 0
+        while f < self.frames and spent < budget_s:
+            for t in range(2):
+                xb = inputs.bits(inputs.rollout_chunk(f, t, heads=self.heads, tokens=self.tokens))
+                t1 = time.perf_counter()
+                caches[t].append(f * self.rpc, xb, self.rule)
+                caches[t].dequantize(0, (f + 1) * self.rpc)
+                spent += time.perf_counter() - t1
+                nbytes += self.chunk_elems * (B_AMAX + B_QUANT) + (f + 1) * self.chunk_elems * B_DEQUANT
+            f += 1
+        return nbytes, spent, f"layer 0 K and V (2 of {2 * self.layers} tensors), frames 1..{f} of the rollout"
+
+
+class Layer:
+    name = "layer"
+
+    def __init__(self, args, rank):
+        self.heads, self.tokens, self.D = 24, 4680, 128
+        if args.small:
+            self.heads, self.tokens = 2, 300
+        self.rule = args.rule or "mse"
+        self.rank = rank
+        self.n = self.heads * self.tokens * self.D
+        self.config = {"workload": f"layer K and V quantize+dequantize: [1,{self.heads},{self.tokens},{self.D}] "
+                                   f"Student-t(3) with 4 outlier channels/head x20, rule {self.rule}",
+                       "model": "Wan-shaped attention layer (synthetic)", "global_batch": 1,
+                       "seq_len": self.tokens, "parallelism": "replica per GPU",
+                       "l2": "flushed between timed steps (256 MB write)"}
+        self.flush = True
+
+    def setup(self, kvq, inputs, dev):
+        self.x = [inputs.layer_kv(2 * self.rank + kv, heads=self.heads, tokens=self.tokens, device=dev)
+                  for kv in (0, 1)]
+        self.p = [torch.empty(self.n // 2, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.s = [torch.empty(self.n // 16, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.a = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.y = [torch.empty(self.n, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.kvq = kvq
+
+    def segments(self):
+        kvq = self.kvq
+
+        def q():
+            for i in range(2):
+                kvq.kvq_quantize(self.x[i], self.D, self.rule, amax_out=self.a[i], packed=self.p[i], scales=self.s[i])
+
+        def d():
+            for i in range(2):
+                kvq.kvq_dequantize(self.p[i], self.s[i], self.a[i], self.D, y=self.y[i])
+        return [Segment("quantize", q, 6, 2 * self.n * (B_AMAX + B_QUANT), h2d=tuple(self.x)),
+                Segment("dequant", d, 2, 2 * self.n * B_DEQUANT)]
+
+    def d2h(self):
+        return self.p + self.s + self.a + self.y
+
+    def tokens_per_step(self):
+        return self.tokens
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        nbytes, spent, done = 0.0, 0.0, 0
+        for kv in (0, 1):
+            xb = inputs.bits(inputs.layer_kv(kv, heads=self.heads, tokens=self.tokens))
+            t1 = time.perf_counter()
+            p, s, a = orc.quantize(xb, self.D, self.rule)
+            orc.dequantize(p, s, a, self.D)
+            spent += time.perf_counter() - t1
+            nbytes += self.n * (B_AMAX + B_QUANT + B_DEQUANT)
+            done += 1
+            if spent > budget_s:
+                break
+        return nbytes, spent, f"{done} of 2 tensors (K, V), full size"
+
+
+class Cache:
+    name = "cache"
+
+    def __init__(self, args, rank):
+        self.layers, self.heads, self.tokens, self.D = 30, 24, 32760, 128
+        if args.small:
+            self.layers, self.heads, self.tokens = 2, 2, 2000
+        self.rule = args.rule or "mse"
+        self.rank = rank
+        self.n = self.heads * self.tokens * self.D
+        self.config = {"workload": f"full cache quantize then per-layer dequantize: {self.layers} layers x {{K,V}} x "
+                                   f"[1,{self.heads},{self.tokens},{self.D}], N(0,1) + 1% tokens x10, rule {self.rule}",
+                       "model": "Wan-shaped KV cache (synthetic)", "global_batch": 1, "seq_len": self.tokens,
+                       "parallelism": "replica per GPU", "l2": "inputs larger than L2"}
+
+    def setup(self, kvq, inputs, dev):
+        T = 2 * self.layers
+        self.x = torch.empty((T, self.n), dtype=torch.bfloat16, device=dev)
+        for t in range(T):
+            self.x[t] = inputs.cache_kv(t // 2 + self.layers * self.rank, t % 2, heads=self.heads,
+                                        tokens=self.tokens, device=dev).reshape(-1)
+        self.p = torch.empty((T, self.n // 2), dtype=torch.uint8, device=dev)
+        self.s = torch.empty((T, self.n // 16), dtype=torch.uint8, device=dev)
+        self.a = torch.empty((T, 1), dtype=torch.float32, device=dev)
+        self.y = torch.empty((2, self.n), dtype=torch.bfloat16, device=dev)
+        self.kvq = kvq
+
+    def segments(self):
+        kvq, T = self.kvq, 2 * self.layers
+
+        def q():
+            for t in range(T):
+                kvq.kvq_quantize(self.x[t], self.D, self.rule, amax_out=self.a[t], packed=self.p[t], scales=self.s[t])
+
+        def d():
+            for t in range(T):
+                kvq.kvq_dequantize(self.p[t], self.s[t], self.a[t], self.D, y=self.y[t % 2])
+        return [Segment("quantize", q, 3 * T, T * self.n * (B_AMAX + B_QUANT), h2d=(self.x,)),
+                Segment("dequant", d, T, T * self.n * B_DEQUANT)]
+
+    def d2h(self):
+        return [self.p, self.s, self.a]
+
+    def tokens_per_step(self):
+        return self.tokens
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        spent, nbytes, done = 0.0, 0.0, 0
+        for t in range(2 * self.layers):
+            xb = inputs.bits(inputs.cache_kv(t // 2, t % 2, heads=self.heads, tokens=self.tokens))
+            t1 = time.perf_counter()
+            p, s, a = orc.quantize(xb, self.D, self.rule)
+            orc.dequantize(p, s, a, self.D)
+            spent += time.perf_counter() - t1
+            nbytes += self.n * (B_AMAX + B_QUANT + B_DEQUANT)
+            done += 1
+            if spent > budget_s:
+                break
+        return nbytes, spent, f"{done} of {2 * self.layers} tensors, full size"
+
+
+class Single(Layer):
+    name = "single"
+
+    def __init__(self, args, rank):
+        self.heads, self.tokens, self.D = 1, 4096, 128
+        self.rule = args.rule or "static_6"
+        self.rank = rank
+        self.n = self.tokens * self.D
+        self.config = {"workload": f"single K quantize+dequantize: [4096,128] N(0,1), rule {self.rule}",
+                       "model": "one K tensor (synthetic)", "global_batch": 1, "seq_len": 4096,
+                       "parallelism": "replica per GPU", "l2": "flushed between timed steps (256 MB write)"}
+        self.flush = True
+
+    def setup(self, kvq, inputs, dev):
+        Layer.setup(self, kvq, inputs, dev)
+        self.x = [inputs.normal((self.tokens, self.D), seed=2 * self.rank + kv, device=dev) for kv in (0, 1)]
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        t0, nbytes, reps = time.perf_counter(), 0.0, 0
+        xb = inputs.bits(inputs.single_k())
+        t0 = time.perf_counter()
+        while reps < 2 or time.perf_counter() - t0 < min(budget_s, 5.0):
+            p, s, a = orc.quantize(xb, self.D, self.rule)
+            orc.dequantize(p, s, a, self.D)
+            nbytes += self.n * (B_AMAX + B_QUANT + B_DEQUANT)
+            reps += 1
+        return nbytes, time.perf_counter() - t0, f"[4096,128] K, {reps} repetitions"
+
+
+class Sweep(Layer):
+    name = "sweep"
+
+    def __init__(self, args, rank):
+        self.heads, self.tokens, self.D = 1, args.tokens, 128
+        self.rule = args.rule or "static_6"
+        self.rank = rank
+        self.n = self.tokens * self.D
+        self.flush = self.n * 2 * 2 < L2_BYTES * 4
+        self.config = {"workload": f"sweep quantize+dequantize: [{self.tokens},128] N(0,1), rule {self.rule}",
+                       "model": "bandwidth sweep (synthetic)", "global_batch": 1, "seq_len": self.tokens,
+                       "parallelism": "replica per GPU",
+                       "l2": "flushed between timed steps (256 MB write)" if self.flush else "inputs larger than L2"}
+
+    def setup(self, kvq, inputs, dev):
+        Layer.setup(self, kvq, inputs, dev)
+        self.x = [inputs.sweep(self.tokens, device=dev)] * 2
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        nbytes, reps = 0.0, 0
+        m = min(self.tokens, 1 << 18)
+        xb = inputs.bits(inputs.sweep(self.tokens)[:m])
+        t0 = time.perf_counter()
+        while reps < 1 or time.perf_counter() - t0 < min(budget_s, 5.0):
+            p, s, a = orc.quantize(xb, self.D, self.rule)
+            orc.dequantize(p, s, a, self.D)
+            nbytes += m * self.D * (B_AMAX + B_QUANT + B_DEQUANT)
+            reps += 1
+        return nbytes, time.perf_counter() - t0, f"first {m} of {self.tokens} rows, {reps} repetitions"
+
+
+WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep)}
+
+
+# ---------------------------------------------------------------------------- runner
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(wl, budget_s):
+    import oracle
+    from nvfp4_kv_cache_kvq_b200 import inputs
+
+    oracle.build()
+    nbytes, dt, sample = wl.oracle_sample(oracle, inputs, budget_s)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": oracle.default_threads(), "kind": "oracle",
+            "sample": sample, "seconds": round(dt, 3)}
+
+
+def run_reference(args, wl, world, rank):
+    """The CPU oracle, as it stands, on a bounded sample of the workload per step."""
+    if rank != 0:
+        return
+    import oracle
+    from nvfp4_kv_cache_kvq_b200 import inputs
+
+    oracle.build()
+    per_step = []
+    sample = ""
+    for i in range(args.warmup + args.steps):
+        nbytes, dt, sample = wl.oracle_sample(oracle, inputs, args.ref_step_s)
+        if i >= args.warmup:
+            per_step.append((nbytes, dt))
+    tot_b = sum(b for b, _ in per_step)
+    tot_t = sum(t for _, t in per_step)
+    value = tot_b / tot_t / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / len(per_step), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": wl.config,
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.default_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def capture(segs, use_graphs):
+    if not use_graphs:
+        return
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for seg in segs:  # one eager run first: builds the library and settles its queries
+            seg.fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for seg in segs:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            seg.fn()
+        seg.graph = g
+    torch.cuda.synchronize()
+
+
+def run_step(segs, events, e2e=None):
+    """One bench step on the current stream; events[i] is recorded before segment i and
+    events[-1] after the last. With e2e, every segment's inputs are first copied in
+    from pinned host memory (inside its event interval)."""
+    for i, seg in enumerate(segs):
+        events[i].record()
+        if e2e is not None and seg.h2d is not None:
+            for dst, src in zip(seg.h2d, e2e["h2d"][i]):
+                dst.copy_(src, non_blocking=True)
+        if seg.graph is not None:
+            seg.graph.replay()
+        else:
+            seg.fn()
+    if e2e is not None:
+        for dst, src in zip(e2e["d2h_dst"], e2e["d2h_src"]):
+            dst.copy_(src, non_blocking=True)
+    events[-1].record()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="rollout")
+    ap.add_argument("--rule", choices=("static_6", "static_4", "mse"), default=None)
+    ap.add_argument("--tokens", type=int, default=1 << 24, help="rows of the sweep workload")
+    ap.add_argument("--small", action="store_true", help="a reduced shape of the workload (for tests)")
+    ap.add_argument("--no-graphs", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-step-s", type=float, default=8.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores; other ranks exit without work
+        world, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
+        run_reference(args, WORKLOADS[args.workload](args, rank), world, rank)
+        return
+    world, rank, _ = dist_setup()
+    wl = WORKLOADS[args.workload](args, rank)
+
+    import nvfp4_kv_cache_kvq_b200 as kvq
+    from nvfp4_kv_cache_kvq_b200 import inputs
+
+    kvq.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl.setup(kvq, inputs, dev)
+    segs = wl.segments()
+    capture(segs, not args.no_graphs)
+    flush_buf = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev) if getattr(wl, "flush", False) else None
+
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(len(segs) + 1)]
+    for _ in range(args.warmup):
+        run_step(segs, events)
+    torch.cuda.synchronize()
+
+    kinds = sorted({s.kind for s in segs})
+    kind_ms = {k: 0.0 for k in kinds}
+    step_ms = []
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        for _ in range(args.steps):
+            if flush_buf is not None:
+                flush_buf.zero_()
+            run_step(segs, events)
+            torch.cuda.synchronize()
+            for i, seg in enumerate(segs):
+                kind_ms[seg.kind] += events[i].elapsed_time(events[i + 1])
+            step_ms.append(events[0].elapsed_time(events[-1]))
+    torch.cuda.synchronize()
+    barrier(world)
+    mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+
+    bytes_step = sum(s.bytes_alg for s in segs)
+    value = world * bytes_step / (mean_ms * 1e-3) / 1e9
+    peak, peak_src = peaks()
+    kind_bytes = {k: sum(s.bytes_alg for s in segs if s.kind == k) for k in kinds}
+    kind_launch = {k: sum(s.launches for s in segs if s.kind == k) for k in kinds}
+    dom = max(kinds, key=lambda k: kind_ms[k])
+    dom_ms = kind_ms[dom] / args.steps
+    achieved = kind_bytes[dom] / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "traffic": None, "launches_per_step": kind_launch[dom],
+                "alg_bytes_per_step": kind_bytes[dom], "ms_per_step": dom_ms}
+    per_kind = {k: {"ms_per_step": kind_ms[k] / args.steps,
+                    "GB_s": kind_bytes[k] / (kind_ms[k] / args.steps * 1e-3) / 1e9 if kind_ms[k] else None,
+                    "launches_per_step": kind_launch[k]} for k in kinds}
+
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": mean_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": wl.config,
+            "hbm_frac": value / world / peak, "tokens_per_s": world * wl.tokens_per_step() / (mean_ms * 1e-3),
+            "roofline": roofline, "kernels": per_kind, "gpu_launches": sum(s.launches for s in segs) * args.steps,
+            "clocks": sampler.summary(), "graphs": not args.no_graphs}
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, wl, segs, bytes_step, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        for s in segs:
+            s.graph = None
+        dist.destroy_process_group()
+
+
+def run_e2e(args, wl, segs, bytes_step, world):
+    """The same steps with every segment's inputs copied in from pinned host memory and
+    the step's outputs copied back, inside the timed region."""
+    h2d, h2d_bytes = [], 0
+    for seg in segs:
+        if seg.h2d is None:
+            h2d.append(None)
+            continue
+        srcs = []
+        for t in seg.h2d:
+            host = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            host.copy_(t)
+            srcs.append(host)
+            h2d_bytes += t.numel() * t.element_size()
+        h2d.append(srcs)
+    d2h_src = wl.d2h()
+    d2h_dst = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d2h_src]
+    d2h_bytes = sum(t.numel() * t.element_size() for t in d2h_src)
+    e2e = {"h2d": h2d, "d2h_src": d2h_src, "d2h_dst": d2h_dst}
+    events = [torch.cuda.Event(enable_timing=True) for _ in range(len(segs) + 1)]
+    run_step(segs, events, e2e)
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    ms = []
+    for _ in range(steps):
+        run_step(segs, events, e2e)
+        torch.cuda.synchronize()
+        ms.append(events[0].elapsed_time(events[-1]))
+    mean_ms = max_over_ranks(sum(ms) / len(ms), world)
+    return {"value": world * bytes_step / (mean_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": mean_ms,
+            "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "steps": steps}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+/*
+ * kvq.h -- C ABI of libkvq: blockwise NVFP4 quantization of attention K/V caches on
+ * NVIDIA B200 (sm_100a), and dequantization back to bf16.
+ *
+ * Format (the pages' method, restated):
+ *   - A tensor is a flat array of bf16 rows of head_dim elements. Every 16 consecutive
+ *     elements of a row form a block.
+ *   - Each element is stored as an FP4 e2m1 code (sign, 2 exponent bits, 1 mantissa
+ *     bit; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6), two codes per byte, the even element
+ *     in the low nibble ("How NVFP4 Quantization Works in LongLive 2.0 for Transformer
+ *     Inference", section "Stage 1: Weight Quantization", step 3).
+ *   - Each block has one FP8 e4m3 scale byte ("Understanding the NVFP4 Format and
+ *     Architecture": block scales quantized to FP8).
+ *   - Each tensor (or each appended chunk of a cache) has one fp32 amax. Its global
+ *     scale is gs = amax / (6 * 448) ("Stage 3: KV-Cache De-quantization at
+ *     Inference", step 3).
+ *
+ * Quantization of one block, with amax_b = max |x| over the block and a denominator
+ * R (6 for static_6, 4 for static_4; rule mse tries both):
+ *     c   = e4m3_rne_satfinite((amax_b / R) / gs)        (c = 0 when gs == 0)
+ *     S   = e4m3_value(c) * gs
+ *     inv = 1 / S, replaced by 0 when it is infinite
+ *     q_i = e2m1_rne_satfinite(x_i * inv)                 (sign kept, also for zero)
+ *   Rule mse keeps R = 4 only when its squared error is strictly smaller. The error is
+ *   the sum of (x_i - value(q_i) * S)^2, each residual one fused multiply-add, the squares
+ *   accumulated by fused multiply-add into an even-position and an odd-position partial
+ *   sum (index order), which are then added. All arithmetic is IEEE fp32,
+ *   round-to-nearest-even. ("How to Use KV Cache Quantization with LongLive's
+ *   LongLiveQuantizationConfig", section "Configuration Parameters Reference": scale
+ *   rules static_6, static_4 and mse.)
+ * Dequantization: y_i = bf16_rne(value(q_i) * S), the product rounded to fp32 first
+ * ("CUDA De-quantization Pipeline"; "Stage 3", steps 2-3).
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" are CUDA device (or managed) memory that the caller
+ *     allocates, owns and frees. The library never allocates or frees memory and keeps
+ *     no state between calls. Host pointers are read before the call returns.
+ *   - Work is queued on `stream` (a cudaStream_t; NULL is the legacy default stream)
+ *     and runs asynchronously; results are valid once the stream has been
+ *     synchronized. Calls on the same stream run in order.
+ *   - Arguments are checked on the host before anything is queued. On any error
+ *     nothing is launched and the outputs are untouched (except KVQ_ERR_CUDA, which is
+ *     returned when a launch itself fails). kvq_last_error() describes the last
+ *     failure of the calling thread.
+ *   - Inputs must be finite bf16 (NaN or Inf give unspecified codes). n_elems == 0
+ *     is a valid no-op.
+ *   - Alignment: bf16 tensors (x, y) 32-byte aligned; packed codes 8-byte aligned.
+ *     A misaligned pointer returns KVQ_ERR_MISALIGNED.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without including CUDA headers. */
+typedef struct CUstream_st* kvq_stream_t;
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, unknown rule */
+    KVQ_ERR_MISALIGNED = 2,  /* a pointer below the alignment stated above */
+    KVQ_ERR_UNSUPPORTED = 3, /* a size beyond what the kernels index (see each call) */
+    KVQ_ERR_CAPACITY = 4,    /* a cache range past capacity_rows */
+    KVQ_ERR_CUDA = 5         /* a CUDA runtime error while queuing work */
+} kvq_status;
+
+/* Block-scale rule ("Configuration Parameters Reference": scale_rule). */
+typedef enum {
+    KVQ_RULE_STATIC_6 = 0, /* scale = amax_b / 6 */
+    KVQ_RULE_STATIC_4 = 1, /* scale = amax_b / 4 */
+    KVQ_RULE_MSE = 2       /* per block, the one of the two with the lower squared error */
+} kvq_scale_rule;
+
+/* Largest number of tensors one kvq_*_batch launch covers; larger batches are split
+ * into several launches. */
+#define KVQ_MAX_BATCH 64
+
+/*
+ * kvq_quantize -- quantize one bf16 tensor.
+ *   Defined by "Stage 1: Weight Quantization (FP32 to NVFP4)" steps 1-4 (block amax,
+ *   block scale by the rule, two FP4 values per uint8, a global amax for the tensor)
+ *   and "FP4 Quantization in the Causal Model" (each K and V block quantized on its own).
+ *   x        device, bf16[n_elems], 32-byte aligned. Read only.
+ *   n_elems  number of elements, a multiple of head_dim (at most 2^36).
+ *   head_dim row length, a positive multiple of 16.
+ *   rule     KVQ_RULE_*.
+ *   amax_in  device, 1 float, or NULL. When given, it is used as the tensor amax (the
+ *            caller already knows it and the amax pass is skipped).
+ *   amax_out device, 1 float, or NULL. Receives the amax used (the computed one, or a
+ *            copy of *amax_in). At least one of amax_in / amax_out must be non-NULL.
+ *   packed   device, uint8[n_elems / 2], 8-byte aligned. Written.
+ *   scales   device, uint8[n_elems / 16] (e4m3 codes, one per block, same order). Written.
+ */
+kvq_status kvq_quantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
+                        const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
+                        kvq_stream_t stream);
+
+/*
+ * kvq_dequantize -- the inverse of kvq_quantize, to bf16 ("CUDA De-quantization
+ *   Pipeline": packed cache + scale factors -> bf16; "Stage 3" steps 2-3).
+ *   packed  device, uint8[n_elems / 2], 8-byte aligned.
+ *   scales  device, uint8[n_elems / 16].
+ *   amax    device, 1 float (the amax kvq_quantize wrote).
+ *   y       device, bf16[n_elems], 32-byte aligned. Written; same element order as x.
+ */
+kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const float* amax, int64_t n_elems,
+                          int32_t head_dim, void* y, kvq_stream_t stream);
+
+/*
+ * A packed K or V cache of one layer, in device memory, token-major: row
+ * t * heads + h holds head h of token t, head_dim elements. Rows are grouped in chunks
+ * of rows_per_chunk (one chunk = the rows one append writes, e.g. one latent frame of
+ * 1560 tokens x heads); every chunk has its own amax, written by the append that filled
+ * it ("FP4 Quantization in the Causal Model": every new K/V block is quantized on its
+ * own). kvq_cache_bytes gives the sizes.
+ */
+typedef struct {
+    uint8_t* packed;        /* device, capacity_rows * head_dim / 2 bytes, 8-byte aligned */
+    uint8_t* scales;        /* device, capacity_rows * head_dim / 16 bytes */
+    float* amax;            /* device, ceil(capacity_rows / rows_per_chunk) floats */
+    int64_t capacity_rows;  /* rows the cache holds */
+    int64_t rows_per_chunk; /* rows per append chunk (> 0) */
+    int32_t head_dim;       /* positive multiple of 16 */
+} kvq_cache;
+
+/*
+ * kvq_append -- quantize-on-write: quantize n_rows new rows x into the cache at
+ *   row_offset, with their own amax in cache->amax[row_offset / rows_per_chunk]
+ *   ("KV Cache Quantization for Self-Forcing Video Generation", appendix Table 3:
+ *   quantize-on-write every step, block size 16).
+ *   cache      host pointer to the cache view.
+ *   row_offset first row written; a multiple of rows_per_chunk.
+ *   x          device, bf16[n_rows * head_dim], 32-byte aligned.
+ *   n_rows     0 .. rows_per_chunk; row_offset + n_rows <= capacity_rows
+ *              (else KVQ_ERR_CAPACITY).
+ */
+kvq_status kvq_append(const kvq_cache* cache, int64_t row_offset, const void* x, int64_t n_rows,
+                      kvq_scale_rule rule, kvq_stream_t stream);
+
+/*
+ * kvq_append_batch -- n_tensors appends of the same n_rows in one set of launches
+ *   (e.g. every layer's K and V of one frame).
+ *   caches      host array of n_tensors cache views (same head_dim).
+ *   row_offsets host array of n_tensors row offsets (each a multiple of its
+ *               rows_per_chunk).
+ *   xs          host array of n_tensors device pointers, bf16[n_rows * head_dim] each.
+ *   The tensors must not overlap one another.
+ */
+kvq_status kvq_append_batch(const kvq_cache* caches, const int64_t* row_offsets, const void* const* xs,
+                            int32_t n_tensors, int64_t n_rows, kvq_scale_rule rule, kvq_stream_t stream);
+
+/*
+ * kvq_dequantize_cache -- dequantize cache rows [row_begin, row_end) to bf16, each row
+ *   with the amax of its chunk ("Stage 3: KV-Cache De-quantization at Inference";
+ *   appendix Table 3: dequantize the active cache back to dense BF16 before attention).
+ *   y  device, bf16[(row_end - row_begin) * head_dim], 32-byte aligned. Written.
+ *   row_end <= capacity_rows (else KVQ_ERR_CAPACITY).
+ */
+kvq_status kvq_dequantize_cache(const kvq_cache* cache, int64_t row_begin, int64_t row_end, void* y,
+                                kvq_stream_t stream);
+
+/*
+ * kvq_dequantize_cache_batch -- the same row range of n_tensors caches (same head_dim)
+ *   into n_tensors outputs, in one set of launches.
+ *   ys  host array of n_tensors device pointers.
+ */
+kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, int32_t n_tensors,
+                                      int64_t row_begin, int64_t row_end, kvq_stream_t stream);
+
+/*
+ * kvq_cache_bytes -- host only. Bytes of a cache of `layers` layers x {K, V}, each
+ *   capacity_tokens x heads rows of head_dim, chunks of tokens_per_chunk tokens:
+ *     packed = 2*layers * capacity_tokens*heads*head_dim / 2
+ *     scales = 2*layers * capacity_tokens*heads*head_dim / 16
+ *     amax   = 2*layers * ceil(capacity_tokens / tokens_per_chunk) * 4
+ *   (4.5 bits per element plus one float per chunk: "How NVFP4 Quantization Works",
+ *   FAQ on memory savings; Self-Forcing study, Figure 6, compressed versus
+ *   BF16-equivalent footprint). Any output pointer may be NULL.
+ */
+kvq_status kvq_cache_bytes(int32_t layers, int32_t heads, int64_t capacity_tokens, int32_t head_dim,
+                           int64_t tokens_per_chunk, uint64_t* packed_bytes, uint64_t* scale_bytes,
+                           uint64_t* amax_bytes);
+
+/* Human-readable name of a status code (static string). */
+const char* kvq_status_string(kvq_status status);
+
+/* Description of the last error returned to the calling thread ("" if none). */
+const char* kvq_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

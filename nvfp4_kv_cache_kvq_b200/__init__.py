@@ -1,0 +1,236 @@
+"""nvfp4_kv_cache_kvq_b200 -- blockwise NVFP4 KV-cache quantization for B200.
+
+Thin Python binding of ``libkvq.so`` (C ABI in ``include/kvq.h``). The functions here
+carry the C names and only marshal arguments: torch tensors become device pointers,
+the current torch CUDA stream becomes the ``cudaStream_t``, and missing outputs are
+allocated with torch. Every step of the computation runs in the library's CUDA kernels;
+there is no other code path. Loading fails loudly when the library cannot be built or
+loaded.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+BLOCK = 16
+RULES = {"static_6": 0, "static_4": 1, "mse": 2}
+STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_MISALIGNED", 3: "KVQ_ERR_UNSUPPORTED",
+          4: "KVQ_ERR_CAPACITY", 5: "KVQ_ERR_CUDA"}
+MAX_BATCH = 64
+
+_lib = None
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("amax", ctypes.c_void_p),
+                ("capacity_rows", ctypes.c_int64), ("rows_per_chunk", ctypes.c_int64),
+                ("head_dim", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load() -> ctypes.CDLL:
+    """Build (if stale) and load libkvq.so. Raises if either step fails."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.build()
+    lib = ctypes.CDLL(path)
+    P, I64, I32, U64P = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint64)
+    CP = ctypes.POINTER(_Cache)
+    sig = {
+        "kvq_quantize": [P, I64, I32, I32, P, P, P, P, P],
+        "kvq_dequantize": [P, P, P, I64, I32, P, P],
+        "kvq_append": [CP, I64, P, I64, I32, P],
+        "kvq_append_batch": [CP, ctypes.POINTER(I64), ctypes.POINTER(P), I32, I64, I32, P],
+        "kvq_dequantize_cache": [CP, I64, I64, P, P],
+        "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
+        "kvq_cache_bytes": [I32, I32, I64, I32, I64, U64P, U64P, U64P],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes, fn.restype = args, ctypes.c_int
+    lib.kvq_status_string.argtypes, lib.kvq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
+    lib.kvq_last_error.argtypes, lib.kvq_last_error.restype = [], ctypes.c_char_p
+    lib.kvq_version.argtypes, lib.kvq_version.restype = [], ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise KvqError(status, load().kvq_last_error().decode())
+
+
+def _rule(rule) -> int:
+    return RULES[rule] if isinstance(rule, str) else int(rule)
+
+
+def _stream(stream, device) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, what: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    return t.data_ptr()
+
+
+def kvq_status_string(status: int) -> str:
+    return load().kvq_status_string(int(status)).decode()
+
+
+def kvq_version() -> str:
+    return load().kvq_version().decode()
+
+
+def kvq_quantize(x: torch.Tensor, head_dim: int | None = None, rule="static_6", amax_in: torch.Tensor | None = None,
+                 amax_out: torch.Tensor | None = None, packed: torch.Tensor | None = None,
+                 scales: torch.Tensor | None = None, stream=None):
+    """Quantize a bf16 tensor. Returns (packed uint8[n/2], scales uint8[n/16], amax float32[1])."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    n = x.numel()
+    head_dim = int(head_dim or x.shape[-1])
+    dev = x.device
+    if packed is None:
+        packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(n // BLOCK, dtype=torch.uint8, device=dev)
+    if amax_out is None and amax_in is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(load().kvq_quantize(_dev(x, "x"), n, head_dim, _rule(rule),
+                               None if amax_in is None else _dev(amax_in, "amax_in"),
+                               None if amax_out is None else _dev(amax_out, "amax_out"),
+                               _dev(packed, "packed"), _dev(scales, "scales"), _stream(stream, dev)))
+    return packed, scales, (amax_out if amax_out is not None else amax_in)
+
+
+def kvq_dequantize(packed: torch.Tensor, scales: torch.Tensor, amax: torch.Tensor, head_dim: int,
+                   y: torch.Tensor | None = None, shape=None, stream=None) -> torch.Tensor:
+    """Dequantize to bf16. ``shape`` (default flat) applies when y is allocated here."""
+    n = packed.numel() * 2
+    dev = packed.device
+    if y is None:
+        y = torch.empty(shape if shape is not None else (n,), dtype=torch.bfloat16, device=dev)
+    if y.dtype != torch.bfloat16 or y.numel() != n:
+        raise ValueError("y must be bfloat16 with 2 * packed.numel() elements")
+    _check(load().kvq_dequantize(_dev(packed, "packed"), _dev(scales, "scales"), _dev(amax, "amax"), n,
+                                 int(head_dim), _dev(y, "y"), _stream(stream, dev)))
+    return y
+
+
+class KVCache:
+    """A packed K or V cache of one layer (token-major rows of head_dim), backed by torch
+    device tensors. ``rows_per_chunk`` is the rows of one append (tokens x heads)."""
+
+    def __init__(self, capacity_rows: int, rows_per_chunk: int, head_dim: int, device="cuda",
+                 packed: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                 amax: torch.Tensor | None = None):
+        self.capacity_rows, self.rows_per_chunk, self.head_dim = int(capacity_rows), int(rows_per_chunk), int(head_dim)
+        n = self.capacity_rows * self.head_dim
+        n_chunks = -(-self.capacity_rows // self.rows_per_chunk)
+        self.packed = packed if packed is not None else torch.zeros(n // 2, dtype=torch.uint8, device=device)
+        self.scales = scales if scales is not None else torch.zeros(n // BLOCK, dtype=torch.uint8, device=device)
+        self.amax = amax if amax is not None else torch.zeros(n_chunks, dtype=torch.float32, device=device)
+        self.device = self.packed.device
+
+    def struct(self) -> _Cache:
+        return _Cache(_dev(self.packed, "packed"), _dev(self.scales, "scales"), _dev(self.amax, "amax"),
+                      self.capacity_rows, self.rows_per_chunk, self.head_dim)
+
+
+def allocate_caches(layers: int, heads: int, capacity_tokens: int, head_dim: int, tokens_per_chunk: int,
+                    device="cuda") -> list[KVCache]:
+    """2 * layers caches (layer l: K = 2l, V = 2l + 1) carved from three device buffers
+    sized by kvq_cache_bytes."""
+    pb, sb, ab = kvq_cache_bytes(layers, heads, capacity_tokens, head_dim, tokens_per_chunk)
+    t = 2 * layers
+    packed = torch.zeros(pb, dtype=torch.uint8, device=device)
+    scales = torch.zeros(sb, dtype=torch.uint8, device=device)
+    amax = torch.zeros(ab // 4, dtype=torch.float32, device=device)
+    rows = capacity_tokens * heads
+    out = []
+    for i in range(t):
+        out.append(KVCache(rows, tokens_per_chunk * heads, head_dim, device,
+                           packed[i * (pb // t):(i + 1) * (pb // t)], scales[i * (sb // t):(i + 1) * (sb // t)],
+                           amax[i * (ab // 4 // t):(i + 1) * (ab // 4 // t)]))
+    return out
+
+
+def kvq_append(cache: KVCache, row_offset: int, x: torch.Tensor, rule="static_6", stream=None):
+    """Quantize-on-write of x (bf16, n_rows x head_dim) at row_offset of the cache."""
+    c = cache.struct()
+    _check(load().kvq_append(ctypes.byref(c), int(row_offset), _dev(x, "x"), x.numel() // cache.head_dim,
+                             _rule(rule), _stream(stream, cache.device)))
+
+
+def kvq_append_batch(caches, row_offsets, xs, rule="static_6", stream=None):
+    """One append per cache (same row count), in one set of launches."""
+    n = len(caches)
+    if not (len(row_offsets) == len(xs) == n):
+        raise ValueError("caches, row_offsets and xs differ in length")
+    if n == 0:
+        return
+    arr = (_Cache * n)(*[c.struct() for c in caches])
+    offs = (ctypes.c_int64 * n)(*[int(o) for o in row_offsets])
+    ptrs = (ctypes.c_void_p * n)(*[_dev(x, "x") for x in xs])
+    n_rows = xs[0].numel() // caches[0].head_dim
+    if any(x.numel() != xs[0].numel() for x in xs):
+        raise ValueError("all appended tensors must have the same size")
+    _check(load().kvq_append_batch(arr, offs, ptrs, n, n_rows, _rule(rule), _stream(stream, caches[0].device)))
+
+
+def kvq_dequantize_cache(cache: KVCache, row_begin: int, row_end: int, y: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    if y is None:
+        y = torch.empty((row_end - row_begin) * cache.head_dim, dtype=torch.bfloat16, device=cache.device)
+    c = cache.struct()
+    _check(load().kvq_dequantize_cache(ctypes.byref(c), int(row_begin), int(row_end), _dev(y, "y"),
+                                       _stream(stream, cache.device)))
+    return y
+
+
+def kvq_dequantize_cache_batch(caches, row_begin: int, row_end: int, ys=None, stream=None):
+    n = len(caches)
+    if n == 0:
+        return []
+    if ys is None:
+        ys = [torch.empty((row_end - row_begin) * c.head_dim, dtype=torch.bfloat16, device=c.device) for c in caches]
+    arr = (_Cache * n)(*[c.struct() for c in caches])
+    ptrs = (ctypes.c_void_p * n)(*[_dev(y, "y") for y in ys])
+    _check(load().kvq_dequantize_cache_batch(arr, ptrs, n, int(row_begin), int(row_end),
+                                             _stream(stream, caches[0].device)))
+    return ys
+
+
+def kvq_cache_bytes(layers: int, heads: int, capacity_tokens: int, head_dim: int, tokens_per_chunk: int):
+    """(packed bytes, scale bytes, amax bytes) of layers x {K, V}; host only."""
+    p, s, a = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check(load().kvq_cache_bytes(int(layers), int(heads), int(capacity_tokens), int(head_dim),
+                                  int(tokens_per_chunk), ctypes.byref(p), ctypes.byref(s), ctypes.byref(a)))
+    return p.value, s.value, a.value
+
+
+def loaded_library() -> str | None:
+    """Path of the loaded libkvq.so, or None before the first call."""
+    return _build.LIB if _lib is not None else None
+
+
+__all__ = [n for n in dir() if n.startswith("kvq_")] + ["KVCache", "allocate_caches", "KvqError", "load"]

@@ -1,0 +1,733 @@
+// kvq.cu -- libkvq: blockwise NVFP4 KV-cache quantize / dequantize for B200 (sm_100a).
+//
+// The method ("How NVFP4 Quantization Works in LongLive 2.0 for Transformer Inference",
+// sections "Understanding the NVFP4 Format", "Stage 1" and "Stage 3"; "How to Use KV
+// Cache Quantization with LongLive's LongLiveQuantizationConfig", sections "FP4
+// Quantization in the Causal Model", "CUDA De-quantization Pipeline", "Configuration
+// Parameters Reference") is restated in include/kvq.h. This file holds the kernels and
+// the C ABI around them.
+//
+// Kernels (all bandwidth-bound streaming passes; no tensor cores, no shared-memory
+// staging: every access is a fully coalesced 256-bit or narrower vector access):
+//   zero_kernel      clears the amax slots a quantize is about to reduce into.
+//   amax_kernel      max |x| over each tensor: 256-bit loads, per-lane u16x2 max on the
+//                    bf16 bit patterns, warp redux, one atomic max per CTA.
+//   quantize_kernel  one thread per BPT blocks: one 256-bit load per block, block amax,
+//                    e4m3 scale(s) by the rule, e2m1 codes via cvt.satfinite.e2m1x2,
+//                    8 bytes of codes + 1 scale byte per block stored.
+//   dequant_kernel   the mirror image: 8 bytes + 1 scale byte -> one 256-bit bf16 store
+//                    per block; the cache form looks up each block's chunk amax.
+// Every kernel takes a batch of tensors (blockIdx.y = tensor), so one launch covers
+// every layer's K and V of an append or a read.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "kvq.h"
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+constexpr int kBlock = 16;              // elements per quantization block
+constexpr float kGlobalDen = 2688.0f;   // e2m1 max * e4m3 max = 6 * 448
+constexpr int kThreads = 256;
+constexpr int kMaxBatch = KVQ_MAX_BATCH;
+
+// ---------------------------------------------------------------- batch descriptors
+
+struct AmaxBatch {
+    const void* x[kMaxBatch];
+    uint32_t* out[kMaxBatch];  // fp32 amax, reduced as its (non-negative) bit pattern
+    uint64_t n_blocks;
+};
+
+struct ZeroBatch {
+    uint32_t* out[kMaxBatch];
+    int n;
+};
+
+struct QuantTensor {
+    const void* x;
+    uint8_t* packed;
+    uint8_t* scales;
+    const float* amax;  // amax used for this tensor
+    float* amax_copy;   // when non-null, also receives *amax
+};
+
+struct QuantBatch {
+    QuantTensor t[kMaxBatch];
+    uint64_t n_blocks;  // blocks per tensor
+};
+
+struct DequantTensor {
+    const uint8_t* packed;  // at the first block of the range
+    const uint8_t* scales;  // at the first block of the range
+    const float* amax;      // chunk amax array (chunk 0 of the cache) or the tensor amax
+    void* y;
+};
+
+struct DequantBatch {
+    DequantTensor t[kMaxBatch];
+    uint64_t n_blocks;          // blocks per tensor in the range
+    uint64_t block0;            // cache block index of the range's first block
+    uint32_t blocks_per_chunk;  // chunked form only
+};
+
+// ---------------------------------------------------------------- kernels
+
+__global__ void __launch_bounds__(64) zero_kernel(const ZeroBatch z)
+{
+    int i = threadIdx.x;
+    if (i < z.n)
+        *z.out[i] = 0u;
+}
+
+__global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxBatch B)
+{
+    const char* x = static_cast<const char*>(B.x[blockIdx.y]);
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
+    uint64_t b = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    uint32_t m = 0;
+    // four independent 32-byte loads in flight per thread
+    for (; b + 3 * stride < B.n_blocks; b += 4 * stride) {
+        uint32_t w0[8], w1[8], w2[8], w3[8];
+        ld_nc_v8(x + b * 32, w0);
+        ld_nc_v8(x + (b + stride) * 32, w1);
+        ld_nc_v8(x + (b + 2 * stride) * 32, w2);
+        ld_nc_v8(x + (b + 3 * stride) * 32, w3);
+        m = max(m, max(max(block_absmax_bits(w0), block_absmax_bits(w1)),
+                       max(block_absmax_bits(w2), block_absmax_bits(w3))));
+    }
+    for (; b < B.n_blocks; b += stride) {
+        uint32_t w[8];
+        ld_nc_v8(x + b * 32, w);
+        m = max(m, block_absmax_bits(w));
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    __shared__ uint32_t warp_max[kThreads / 32];
+    if ((threadIdx.x & 31) == 0)
+        warp_max[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = threadIdx.x < kThreads / 32 ? warp_max[threadIdx.x] : 0u;
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        if (threadIdx.x == 0 && m != 0u)
+            atomicMax(B.out[blockIdx.y], m << 16);  // bf16 bits -> fp32 bits
+    }
+}
+
+// IEEE reciprocal of a decoded block scale; 0 when it is infinite (S == 0 or S tiny), so
+// that every value of the block is sent to a signed zero.
+__device__ __forceinline__ float safe_rcp(float S)
+{
+    float inv = __frcp_rn(S);
+    return inv == __int_as_float(0x7F800000) ? 0.0f : inv;
+}
+
+// The e2m1 codes of one block under decoded scale reciprocal `inv` (two words).
+__device__ __forceinline__ void encode_values(const float (&x)[kBlock], float inv, uint32_t& q0, uint32_t& q1)
+{
+    float v0[8], v1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v0[i] = __fmul_rn(x[i], inv);
+        v1[i] = __fmul_rn(x[8 + i], inv);
+    }
+    q0 = e2m1x8_from_f32(v0);
+    q1 = e2m1x8_from_f32(v1);
+}
+
+// One mse candidate: the codes of the block under scale S (reciprocal inv) and their
+// squared reconstruction error -- residuals x - value*S by one fma each, squares
+// accumulated by fma into even- and odd-position partial sums, then added.
+__device__ __forceinline__ float encode_values_sq_error(const float (&x)[kBlock], float S, float inv, uint32_t& q0,
+                                                        uint32_t& q1)
+{
+    float v0[8], v1[8], val0[8], val1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v0[i] = __fmul_rn(x[i], inv);
+        v1[i] = __fmul_rn(x[8 + i], inv);
+    }
+    q0 = e2m1x8_encode_decode(v0, val0);
+    q1 = e2m1x8_encode_decode(v1, val1);
+    float se = 0.0f, so = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float de = __fmaf_rn(-val0[i], S, x[i]);
+        const float dodd = __fmaf_rn(-val0[i + 1], S, x[i + 1]);
+        se = __fmaf_rn(de, de, se);
+        so = __fmaf_rn(dodd, dodd, so);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const float de = __fmaf_rn(-val1[i], S, x[8 + i]);
+        const float dodd = __fmaf_rn(-val1[i + 1], S, x[8 + i + 1]);
+        se = __fmaf_rn(de, de, se);
+        so = __fmaf_rn(dodd, dodd, so);
+    }
+    return __fadd_rn(se, so);
+}
+
+// Quantize one block held in w (16 bf16). Returns the scale code; q0/q1 get the codes.
+template <int RULE>
+__device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], float gs, bool gs_zero, uint32_t& q0,
+                                                   uint32_t& q1)
+{
+    const float amax_b = __uint_as_float(block_absmax_bits(w) << 16);
+    float x[kBlock];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        x[2 * j] = bf16lo_to_f32(w[j]);
+        x[2 * j + 1] = bf16hi_to_f32(w[j]);
+    }
+    if (RULE == KVQ_RULE_STATIC_6 || RULE == KVQ_RULE_STATIC_4) {
+        const float s = RULE == KVQ_RULE_STATIC_6 ? __fdiv_rn(amax_b, 6.0f) : __fdiv_rn(amax_b, 4.0f);
+        const float r = __fdiv_rn(s, gs);
+        const uint32_t c = gs_zero ? 0u : (e4m3x2_from_f32(0.0f, r) & 0xFFu);
+        float S, unused;
+        e4m3x2_to_f32(c, S, unused);
+        S = __fmul_rn(S, gs);
+        encode_values(x, safe_rcp(S), q0, q1);
+        return c;
+    } else {
+        const float s6 = __fdiv_rn(amax_b, 6.0f);
+        const float s4 = __fdiv_rn(amax_b, 4.0f);
+        const float r6 = __fdiv_rn(s6, gs);
+        const float r4 = __fdiv_rn(s4, gs);
+        const uint32_t c2 = gs_zero ? 0u : e4m3x2_from_f32(r4, r6);  // c6 in bits 0..7, c4 in 8..15
+        float S6, S4;
+        e4m3x2_to_f32(c2, S6, S4);
+        S6 = __fmul_rn(S6, gs);
+        S4 = __fmul_rn(S4, gs);
+        uint32_t a0, a1, b0, b1;
+        const float e6 = encode_values_sq_error(x, S6, safe_rcp(S6), a0, a1);
+        const float e4 = encode_values_sq_error(x, S4, safe_rcp(S4), b0, b1);
+        const bool use4 = e4 < e6;
+        q0 = use4 ? b0 : a0;
+        q1 = use4 ? b1 : a1;
+        return use4 ? (c2 >> 8) : (c2 & 0xFFu);
+    }
+}
+
+// BPT = blocks per thread per step (1 or 2). With BPT = 2 the packed pointer must be
+// 16-byte aligned and the scale pointer 2-byte aligned.
+template <int RULE, int BPT>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
+{
+    const QuantTensor& T = B.t[blockIdx.y];
+    const float amax = __ldg(T.amax);
+    const float gs = __fdiv_rn(amax, kGlobalDen);
+    const bool gs_zero = gs == 0.0f;
+    if (T.amax_copy != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+        *T.amax_copy = amax;
+
+    const char* x = static_cast<const char*>(T.x);
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
+    const uint64_t n_units = B.n_blocks / BPT;
+    for (uint64_t u = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x; u < n_units; u += stride) {
+        if (BPT == 2) {
+            uint32_t w0[8], w1[8];
+            ld_nc_v8(x + u * 64, w0);
+            ld_nc_v8(x + u * 64 + 32, w1);
+            uint32_t q0, q1, q2, q3;
+            const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, q0, q1);
+            const uint32_t c1 = quantize_block<RULE>(w1, gs, gs_zero, q2, q3);
+            st_v4(T.packed + u * 16, q0, q1, q2, q3);
+            *reinterpret_cast<uint16_t*>(T.scales + u * 2) = static_cast<uint16_t>(c0 | (c1 << 8));
+        } else {
+            uint32_t w0[8];
+            ld_nc_v8(x + u * 32, w0);
+            uint32_t q0, q1;
+            const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, q0, q1);
+            st_v2(T.packed + u * 8, q0, q1);
+            T.scales[u] = static_cast<uint8_t>(c0);
+        }
+    }
+    if (BPT == 2) {  // odd block count: the last block alone
+        const uint64_t b = n_units * 2 + static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+        if (b < B.n_blocks) {
+            uint32_t w0[8];
+            ld_nc_v8(x + b * 32, w0);
+            uint32_t q0, q1;
+            const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, q0, q1);
+            st_v2(T.packed + b * 8, q0, q1);
+            T.scales[b] = static_cast<uint8_t>(c0);
+        }
+    }
+}
+
+// One block: 8 code bytes (two words) and its scale -> 16 bf16 (eight words).
+__device__ __forceinline__ void dequant_block(uint32_t q0, uint32_t q1, uint32_t c, float gs, uint32_t (&y)[8])
+{
+    float S, unused;
+    e4m3x2_to_f32(c & 0xFFu, S, unused);
+    S = __fmul_rn(S, gs);
+    float v[8];
+    e2m1x8_to_f32(q0, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        y[j] = bf16x2_from_f32(__fmul_rn(v[2 * j + 1], S), __fmul_rn(v[2 * j], S));
+    e2m1x8_to_f32(q1, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        y[4 + j] = bf16x2_from_f32(__fmul_rn(v[2 * j + 1], S), __fmul_rn(v[2 * j], S));
+}
+
+template <bool CHUNKED>
+__device__ __forceinline__ float block_gs(const DequantTensor& T, const DequantBatch& B, uint64_t b, float gs_tensor)
+{
+    if (!CHUNKED)
+        return gs_tensor;
+    const uint32_t chunk = static_cast<uint32_t>((B.block0 + b) / B.blocks_per_chunk);
+    return __fdiv_rn(__ldg(T.amax + chunk), kGlobalDen);
+}
+
+template <int BPT, bool CHUNKED>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantBatch B)
+{
+    const DequantTensor& T = B.t[blockIdx.y];
+    const float gs_tensor = CHUNKED ? 0.0f : __fdiv_rn(__ldg(T.amax), kGlobalDen);
+    char* y = static_cast<char*>(T.y);
+    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
+    const uint64_t n_units = B.n_blocks / BPT;
+    for (uint64_t u = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x; u < n_units; u += stride) {
+        if (BPT == 2) {
+            const uint4 q = ld_nc_v4(T.packed + u * 16);
+            const uint32_t c = __ldg(reinterpret_cast<const uint16_t*>(T.scales) + u);
+            uint32_t y0[8], y1[8];
+            dequant_block(q.x, q.y, c, block_gs<CHUNKED>(T, B, 2 * u, gs_tensor), y0);
+            dequant_block(q.z, q.w, c >> 8, block_gs<CHUNKED>(T, B, 2 * u + 1, gs_tensor), y1);
+            st_v8(y + u * 64, y0);
+            st_v8(y + u * 64 + 32, y1);
+        } else {
+            const uint2 q = ld_nc_v2(T.packed + u * 8);
+            const uint32_t c = __ldg(T.scales + u);
+            uint32_t y0[8];
+            dequant_block(q.x, q.y, c, block_gs<CHUNKED>(T, B, u, gs_tensor), y0);
+            st_v8(y + u * 32, y0);
+        }
+    }
+    if (BPT == 2) {
+        const uint64_t b = n_units * 2 + static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+        if (b < B.n_blocks) {
+            const uint2 q = ld_nc_v2(T.packed + b * 8);
+            const uint32_t c = __ldg(T.scales + b);
+            uint32_t y0[8];
+            dequant_block(q.x, q.y, c, block_gs<CHUNKED>(T, B, b, gs_tensor), y0);
+            st_v8(y + b * 32, y0);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+thread_local char g_last_error[512] = "";
+
+kvq_status fail(kvq_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+kvq_status fail(kvq_status st, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+kvq_status ok()
+{
+    g_last_error[0] = '\0';
+    return KVQ_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+kvq_status check_launch(const char* what)
+{
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return KVQ_OK;
+}
+
+// CTAs per tensor for a grid-stride kernel: enough to fill every SM at the kernel's
+// occupancy, spread over the tensors of the batch, and no more than the work needs.
+template <typename K>
+kvq_status grid_x(K kernel, uint64_t units_per_tensor, int n_tensors, unsigned* gx)
+{
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess) {
+        cudaError_t e = cudaGetLastError();
+        return fail(KVQ_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
+    }
+    uint64_t full = static_cast<uint64_t>(sms) * static_cast<uint64_t>(per_sm > 0 ? per_sm : 1);
+    uint64_t want = (full + n_tensors - 1) / n_tensors;
+    uint64_t need = (units_per_tensor + kThreads - 1) / kThreads;
+    uint64_t g = want < need ? want : need;
+    *gx = static_cast<unsigned>(g < 1 ? 1 : g);
+    return KVQ_OK;
+}
+
+kvq_status check_rule(kvq_scale_rule rule)
+{
+    if (rule != KVQ_RULE_STATIC_6 && rule != KVQ_RULE_STATIC_4 && rule != KVQ_RULE_MSE)
+        return fail(KVQ_ERR_INVALID_ARG, "unknown scale rule %d", static_cast<int>(rule));
+    return KVQ_OK;
+}
+
+constexpr uint64_t kMaxElems = 1ull << 36;
+
+kvq_status check_shape(int64_t n_elems, int32_t head_dim)
+{
+    if (head_dim <= 0 || head_dim % kBlock != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "head_dim %d is not a positive multiple of 16", head_dim);
+    if (n_elems < 0 || n_elems % head_dim != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "n_elems %lld is not a non-negative multiple of head_dim %d",
+                    static_cast<long long>(n_elems), head_dim);
+    if (static_cast<uint64_t>(n_elems) > kMaxElems)
+        return fail(KVQ_ERR_UNSUPPORTED, "n_elems %lld above 2^36", static_cast<long long>(n_elems));
+    return KVQ_OK;
+}
+
+// Quantize a batch of equally sized tensors whose amax slots are given. When
+// compute_amax, the slots are cleared and reduced first.
+kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s)
+{
+    if (n == 0 || qb.n_blocks == 0)
+        return KVQ_OK;
+    if (compute_amax) {
+        ZeroBatch z{};
+        AmaxBatch ab{};
+        for (int i = 0; i < n; ++i) {
+            z.out[i] = reinterpret_cast<uint32_t*>(const_cast<float*>(qb.t[i].amax));
+            ab.x[i] = qb.t[i].x;
+            ab.out[i] = z.out[i];
+        }
+        z.n = n;
+        ab.n_blocks = qb.n_blocks;
+        zero_kernel<<<1, 64, 0, s>>>(z);
+        kvq_status st = check_launch("zero_kernel");
+        if (st != KVQ_OK)
+            return st;
+        unsigned gx;
+        if ((st = grid_x(amax_kernel, qb.n_blocks, n, &gx)) != KVQ_OK)
+            return st;
+        amax_kernel<<<dim3(gx, n), kThreads, 0, s>>>(ab);
+        if ((st = check_launch("amax_kernel")) != KVQ_OK)
+            return st;
+    }
+    bool pairs = qb.n_blocks >= 2;
+    for (int i = 0; i < n; ++i)
+        pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
+    const uint64_t units = pairs ? qb.n_blocks / 2 : qb.n_blocks;
+    unsigned gx;
+    kvq_status st;
+#define KVQ_LAUNCH_Q(R, BPT)                                                        \
+    do {                                                                            \
+        if ((st = grid_x(quantize_kernel<R, BPT>, units, n, &gx)) != KVQ_OK)        \
+            return st;                                                              \
+        quantize_kernel<R, BPT><<<dim3(gx, n), kThreads, 0, s>>>(qb);               \
+    } while (0)
+    if (pairs) {
+        if (rule == KVQ_RULE_STATIC_6)
+            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_6, 2);
+        else if (rule == KVQ_RULE_STATIC_4)
+            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_4, 2);
+        else
+            KVQ_LAUNCH_Q(KVQ_RULE_MSE, 2);
+    } else {
+        if (rule == KVQ_RULE_STATIC_6)
+            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_6, 1);
+        else if (rule == KVQ_RULE_STATIC_4)
+            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_4, 1);
+        else
+            KVQ_LAUNCH_Q(KVQ_RULE_MSE, 1);
+    }
+#undef KVQ_LAUNCH_Q
+    return check_launch("quantize_kernel");
+}
+
+kvq_status run_dequantize(const DequantBatch& db, int n, bool chunked, cudaStream_t s)
+{
+    if (n == 0 || db.n_blocks == 0)
+        return KVQ_OK;
+    bool pairs = db.n_blocks >= 2;
+    for (int i = 0; i < n; ++i)
+        pairs = pairs && aligned(db.t[i].packed, 16) && aligned(db.t[i].scales, 2);
+    const uint64_t units = pairs ? db.n_blocks / 2 : db.n_blocks;
+    unsigned gx;
+    kvq_status st;
+#define KVQ_LAUNCH_D(BPT, CH)                                                     \
+    do {                                                                          \
+        if ((st = grid_x(dequant_kernel<BPT, CH>, units, n, &gx)) != KVQ_OK)      \
+            return st;                                                            \
+        dequant_kernel<BPT, CH><<<dim3(gx, n), kThreads, 0, s>>>(db);             \
+    } while (0)
+    if (pairs) {
+        if (chunked)
+            KVQ_LAUNCH_D(2, true);
+        else
+            KVQ_LAUNCH_D(2, false);
+    } else {
+        if (chunked)
+            KVQ_LAUNCH_D(1, true);
+        else
+            KVQ_LAUNCH_D(1, false);
+    }
+#undef KVQ_LAUNCH_D
+    return check_launch("dequant_kernel");
+}
+
+kvq_status check_cache(const kvq_cache* c, const char* what)
+{
+    if (c == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: null cache", what);
+    if (c->head_dim <= 0 || c->head_dim % kBlock != 0)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: head_dim %d is not a positive multiple of 16", what, c->head_dim);
+    if (c->rows_per_chunk <= 0 || c->capacity_rows < 0)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: bad rows_per_chunk / capacity_rows", what);
+    if (c->packed == nullptr || c->scales == nullptr || c->amax == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: null cache buffer", what);
+    if (!aligned(c->packed, 8) || !aligned(c->amax, 4))
+        return fail(KVQ_ERR_MISALIGNED, "%s: cache packed must be 8-byte and amax 4-byte aligned", what);
+    const uint64_t elems = static_cast<uint64_t>(c->capacity_rows) * static_cast<uint64_t>(c->head_dim);
+    if (elems > kMaxElems)
+        return fail(KVQ_ERR_UNSUPPORTED, "%s: cache above 2^36 elements", what);
+    const uint64_t bpc = static_cast<uint64_t>(c->rows_per_chunk) * static_cast<uint64_t>(c->head_dim / kBlock);
+    if (bpc > 0xFFFFFFFFull)
+        return fail(KVQ_ERR_UNSUPPORTED, "%s: chunk above 2^32 blocks", what);
+    return KVQ_OK;
+}
+
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+kvq_status kvq_quantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
+                        const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
+                        kvq_stream_t stream)
+{
+    kvq_status st;
+    if ((st = check_shape(n_elems, head_dim)) != KVQ_OK || (st = check_rule(rule)) != KVQ_OK)
+        return st;
+    if (amax_in == nullptr && amax_out == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize: amax_in and amax_out are both null");
+    if (n_elems > 0 && (x == nullptr || packed == nullptr || scales == nullptr))
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize: null tensor pointer");
+    if (!aligned(x, 32) || !aligned(packed, 8) || !aligned(amax_in, 4) || !aligned(amax_out, 4))
+        return fail(KVQ_ERR_MISALIGNED, "kvq_quantize: x must be 32-byte, packed 8-byte, amax 4-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (n_elems == 0) {
+        // amax of an empty tensor is 0; a given amax is passed through
+        if (amax_out != nullptr) {
+            cudaError_t e = amax_in ? cudaMemcpyAsync(amax_out, amax_in, 4, cudaMemcpyDeviceToDevice, s)
+                                    : cudaMemsetAsync(amax_out, 0, 4, s);
+            if (e != cudaSuccess)
+                return fail(KVQ_ERR_CUDA, "kvq_quantize: %s", cudaGetErrorString(e));
+        }
+        return ok();
+    }
+    QuantBatch qb{};
+    qb.n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
+    qb.t[0].x = x;
+    qb.t[0].packed = packed;
+    qb.t[0].scales = scales;
+    qb.t[0].amax = amax_in ? amax_in : amax_out;
+    qb.t[0].amax_copy = (amax_in && amax_out && amax_out != amax_in) ? amax_out : nullptr;
+    if ((st = run_quantize(qb, 1, amax_in == nullptr, rule, s)) != KVQ_OK)
+        return st;
+    return ok();
+}
+
+kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const float* amax, int64_t n_elems,
+                          int32_t head_dim, void* y, kvq_stream_t stream)
+{
+    kvq_status st;
+    if ((st = check_shape(n_elems, head_dim)) != KVQ_OK)
+        return st;
+    if (n_elems == 0)
+        return ok();
+    if (packed == nullptr || scales == nullptr || amax == nullptr || y == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize: null pointer");
+    if (!aligned(y, 32) || !aligned(packed, 8) || !aligned(amax, 4))
+        return fail(KVQ_ERR_MISALIGNED, "kvq_dequantize: y must be 32-byte, packed 8-byte, amax 4-byte aligned");
+    DequantBatch db{};
+    db.n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
+    db.t[0].packed = packed;
+    db.t[0].scales = scales;
+    db.t[0].amax = amax;
+    db.t[0].y = y;
+    if ((st = run_dequantize(db, 1, false, reinterpret_cast<cudaStream_t>(stream))) != KVQ_OK)
+        return st;
+    return ok();
+}
+
+kvq_status kvq_append_batch(const kvq_cache* caches, const int64_t* row_offsets, const void* const* xs,
+                            int32_t n_tensors, int64_t n_rows, kvq_scale_rule rule, kvq_stream_t stream)
+{
+    kvq_status st;
+    if ((st = check_rule(rule)) != KVQ_OK)
+        return st;
+    if (n_tensors < 0 || n_rows < 0)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_append_batch: negative count");
+    if (n_tensors == 0)
+        return ok();
+    if (caches == nullptr || row_offsets == nullptr || xs == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_append_batch: null host array");
+    const int32_t D = caches[0].head_dim;
+    for (int i = 0; i < n_tensors; ++i) {
+        const kvq_cache* c = &caches[i];
+        if ((st = check_cache(c, "kvq_append")) != KVQ_OK)
+            return st;
+        if (c->head_dim != D)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_append_batch: head_dim differs between tensors");
+        const int64_t off = row_offsets[i];
+        if (off < 0 || off % c->rows_per_chunk != 0)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_append: row_offset %lld is not a non-negative multiple of "
+                        "rows_per_chunk %lld", static_cast<long long>(off), static_cast<long long>(c->rows_per_chunk));
+        if (n_rows > c->rows_per_chunk)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_append: n_rows %lld exceeds rows_per_chunk %lld",
+                        static_cast<long long>(n_rows), static_cast<long long>(c->rows_per_chunk));
+        if (off > c->capacity_rows - n_rows)
+            return fail(KVQ_ERR_CAPACITY, "kvq_append: rows [%lld, %lld) past capacity %lld",
+                        static_cast<long long>(off), static_cast<long long>(off + n_rows),
+                        static_cast<long long>(c->capacity_rows));
+        if (n_rows > 0 && xs[i] == nullptr)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_append: null x");
+        if (!aligned(xs[i], 32))
+            return fail(KVQ_ERR_MISALIGNED, "kvq_append: x must be 32-byte aligned");
+    }
+    if (n_rows == 0)
+        return ok();
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const uint64_t n_blocks = static_cast<uint64_t>(n_rows) * static_cast<uint64_t>(D / kBlock);
+    for (int base = 0; base < n_tensors; base += kMaxBatch) {
+        const int n = n_tensors - base < kMaxBatch ? n_tensors - base : kMaxBatch;
+        QuantBatch qb{};
+        qb.n_blocks = n_blocks;
+        for (int i = 0; i < n; ++i) {
+            const kvq_cache* c = &caches[base + i];
+            const int64_t off = row_offsets[base + i];
+            const uint64_t e0 = static_cast<uint64_t>(off) * static_cast<uint64_t>(D);
+            qb.t[i].x = xs[base + i];
+            qb.t[i].packed = c->packed + e0 / 2;
+            qb.t[i].scales = c->scales + e0 / kBlock;
+            qb.t[i].amax = c->amax + off / c->rows_per_chunk;
+            qb.t[i].amax_copy = nullptr;
+        }
+        if ((st = run_quantize(qb, n, true, rule, s)) != KVQ_OK)
+            return st;
+    }
+    return ok();
+}
+
+kvq_status kvq_append(const kvq_cache* cache, int64_t row_offset, const void* x, int64_t n_rows,
+                      kvq_scale_rule rule, kvq_stream_t stream)
+{
+    return kvq_append_batch(cache, &row_offset, &x, 1, n_rows, rule, stream);
+}
+
+kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, int32_t n_tensors,
+                                      int64_t row_begin, int64_t row_end, kvq_stream_t stream)
+{
+    kvq_status st;
+    if (n_tensors < 0)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize_cache_batch: negative count");
+    if (n_tensors == 0)
+        return ok();
+    if (caches == nullptr || ys == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize_cache_batch: null host array");
+    if (row_begin < 0 || row_end < row_begin)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize_cache: bad row range [%lld, %lld)",
+                    static_cast<long long>(row_begin), static_cast<long long>(row_end));
+    const int32_t D = caches[0].head_dim;
+    const int64_t rpc = caches[0].rows_per_chunk;
+    for (int i = 0; i < n_tensors; ++i) {
+        const kvq_cache* c = &caches[i];
+        if ((st = check_cache(c, "kvq_dequantize_cache")) != KVQ_OK)
+            return st;
+        if (c->head_dim != D || c->rows_per_chunk != rpc)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize_cache_batch: head_dim / rows_per_chunk differ");
+        if (row_end > c->capacity_rows)
+            return fail(KVQ_ERR_CAPACITY, "kvq_dequantize_cache: row_end %lld past capacity %lld",
+                        static_cast<long long>(row_end), static_cast<long long>(c->capacity_rows));
+        if (row_end > row_begin && ys[i] == nullptr)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize_cache: null y");
+        if (!aligned(ys[i], 32))
+            return fail(KVQ_ERR_MISALIGNED, "kvq_dequantize_cache: y must be 32-byte aligned");
+    }
+    if (row_end == row_begin)
+        return ok();
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const uint64_t bpr = static_cast<uint64_t>(D / kBlock);
+    for (int base = 0; base < n_tensors; base += kMaxBatch) {
+        const int n = n_tensors - base < kMaxBatch ? n_tensors - base : kMaxBatch;
+        DequantBatch db{};
+        db.n_blocks = static_cast<uint64_t>(row_end - row_begin) * bpr;
+        db.block0 = static_cast<uint64_t>(row_begin) * bpr;
+        db.blocks_per_chunk = static_cast<uint32_t>(static_cast<uint64_t>(rpc) * bpr);
+        for (int i = 0; i < n; ++i) {
+            const kvq_cache* c = &caches[base + i];
+            db.t[i].packed = c->packed + db.block0 * 8;
+            db.t[i].scales = c->scales + db.block0;
+            db.t[i].amax = c->amax;
+            db.t[i].y = ys[base + i];
+        }
+        if ((st = run_dequantize(db, n, true, s)) != KVQ_OK)
+            return st;
+    }
+    return ok();
+}
+
+kvq_status kvq_dequantize_cache(const kvq_cache* cache, int64_t row_begin, int64_t row_end, void* y,
+                                kvq_stream_t stream)
+{
+    return kvq_dequantize_cache_batch(cache, &y, 1, row_begin, row_end, stream);
+}
+
+kvq_status kvq_cache_bytes(int32_t layers, int32_t heads, int64_t capacity_tokens, int32_t head_dim,
+                           int64_t tokens_per_chunk, uint64_t* packed_bytes, uint64_t* scale_bytes,
+                           uint64_t* amax_bytes)
+{
+    if (layers <= 0 || heads <= 0 || capacity_tokens < 0 || head_dim <= 0 || head_dim % kBlock != 0 ||
+        tokens_per_chunk <= 0)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_cache_bytes: bad dimensions");
+    const uint64_t tensors = 2ull * static_cast<uint64_t>(layers);
+    const uint64_t elems = static_cast<uint64_t>(capacity_tokens) * static_cast<uint64_t>(heads) *
+                           static_cast<uint64_t>(head_dim);
+    const uint64_t chunks = (static_cast<uint64_t>(capacity_tokens) + static_cast<uint64_t>(tokens_per_chunk) - 1) /
+                            static_cast<uint64_t>(tokens_per_chunk);
+    if (packed_bytes)
+        *packed_bytes = tensors * (elems / 2);
+    if (scale_bytes)
+        *scale_bytes = tensors * (elems / kBlock);
+    if (amax_bytes)
+        *amax_bytes = tensors * chunks * sizeof(float);
+    return ok();
+}
+
+const char* kvq_status_string(kvq_status status)
+{
+    switch (status) {
+    case KVQ_OK: return "KVQ_OK";
+    case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+    case KVQ_ERR_MISALIGNED: return "KVQ_ERR_MISALIGNED";
+    case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+    case KVQ_ERR_CAPACITY: return "KVQ_ERR_CAPACITY";
+    case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+    }
+    return "KVQ_ERR_UNKNOWN";
+}
+
+const char* kvq_last_error(void) { return g_last_error; }
+
+const char* kvq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

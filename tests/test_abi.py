@@ -1,0 +1,110 @@
+"""The C ABI without a GPU: the library builds for sm_100a, loads, exports every
+function include/kvq.h declares, and rejects bad arguments on the host (before any CUDA
+call). No kernel runs here."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import nvfp4_kv_cache_kvq_b200 as kvq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(kvq_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("kvq_quantize", "kvq_dequantize", "kvq_append", "kvq_append_batch", "kvq_dequantize_cache",
+                 "kvq_dequantize_cache_batch", "kvq_cache_bytes", "kvq_status_string", "kvq_last_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = kvq.load()
+    out = subprocess.check_output(["nm", "-D", "--defined-only", kvq.library_path()], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_library_is_built_for_sm100a_only():
+    from nvfp4_kv_cache_kvq_b200 import build
+
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1 and "-fmad=false" in flags
+
+
+def test_host_only_calls():
+    assert kvq.kvq_status_string(0) == "KVQ_OK"
+    assert kvq.kvq_status_string(4) == "KVQ_ERR_CAPACITY"
+    assert kvq.kvq_version().count(".") == 2
+    p, s, a = kvq.kvq_cache_bytes(30, 12, 93600, 128, 1560)
+    elems = 60 * 93600 * 12 * 128
+    assert (p, s, a) == (elems // 2, elems // 16, 60 * 60 * 4)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_cache_bytes(30, 12, 93600, 100, 1560)
+    assert e.value.status == 1
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_invalid_arguments_rejected_before_any_launch():
+    lib = kvq.load()
+    A = 1 << 40  # never dereferenced: every call below fails validation first
+    # head_dim not a multiple of 16
+    assert lib.kvq_quantize(_fake(A), 96, 12, 0, None, _fake(A), _fake(A), _fake(A), None) == 1
+    # n_elems not a multiple of head_dim
+    assert lib.kvq_quantize(_fake(A), 100, 16, 0, None, _fake(A), _fake(A), _fake(A), None) == 1
+    # unknown rule
+    assert lib.kvq_quantize(_fake(A), 128, 128, 7, None, _fake(A), _fake(A), _fake(A), None) == 1
+    # no amax destination
+    assert lib.kvq_quantize(_fake(A), 128, 128, 0, None, None, _fake(A), _fake(A), None) == 1
+    assert b"both null" in lib.kvq_last_error()
+    # misaligned x / packed / y
+    assert lib.kvq_quantize(_fake(A + 16), 128, 128, 0, None, _fake(A), _fake(A), _fake(A), None) == 2
+    assert lib.kvq_quantize(_fake(A), 128, 128, 0, None, _fake(A), _fake(A + 4), _fake(A), None) == 2
+    assert lib.kvq_dequantize(_fake(A), _fake(A), _fake(A), 128, 128, _fake(A + 2), None) == 2
+    # too large
+    assert lib.kvq_quantize(_fake(A), (1 << 37), 128, 0, None, _fake(A), _fake(A), _fake(A), None) == 3
+
+
+def _cache(capacity_rows=64, rows_per_chunk=16, head_dim=128, base=1 << 40):
+    return kvq._Cache(base, base, base, capacity_rows, rows_per_chunk, head_dim)
+
+
+def test_append_capacity_and_alignment_checked_on_host():
+    lib = kvq.load()
+    c = _cache()
+    x = _fake(1 << 41)
+    assert lib.kvq_append(ctypes.byref(c), 8, x, 16, 0, None) == 1      # not chunk aligned
+    assert lib.kvq_append(ctypes.byref(c), 0, x, 17, 0, None) == 1      # more rows than a chunk
+    assert lib.kvq_append(ctypes.byref(c), 64, x, 16, 0, None) == 4     # past capacity
+    assert lib.kvq_append(ctypes.byref(c), 48, x, 16, 3, None) == 1     # bad rule
+    assert lib.kvq_append(ctypes.byref(c), 48, _fake((1 << 41) + 8), 16, 0, None) == 2
+    bad = _cache(head_dim=24)
+    assert lib.kvq_append(ctypes.byref(bad), 0, x, 16, 0, None) == 1
+    y = _fake(1 << 42)
+    assert lib.kvq_dequantize_cache(ctypes.byref(c), 0, 65, y, None) == 4
+    assert lib.kvq_dequantize_cache(ctypes.byref(c), 10, 5, y, None) == 1
+
+
+def test_batch_rejects_mixed_head_dims():
+    lib = kvq.load()
+    arr = (kvq._Cache * 2)(_cache(), _cache(head_dim=64))
+    offs = (ctypes.c_int64 * 2)(0, 0)
+    ptrs = (ctypes.c_void_p * 2)(1 << 41, 1 << 41)
+    assert lib.kvq_append_batch(arr, offs, ptrs, 2, 16, 0, None) == 1
+    ys = (ctypes.c_void_p * 2)(1 << 42, 1 << 42)
+    assert lib.kvq_dequantize_cache_batch(arr, ys, 2, 0, 16, None) == 1

@@ -63,18 +63,24 @@ struct QuantBatch {
 };
 
 struct DequantTensor {
-    const uint8_t* packed;  // at the first block of the range
-    const uint8_t* scales;  // at the first block of the range
-    const float* amax;      // chunk amax array (chunk 0 of the cache) or the tensor amax
-    void* y;
+    const uint8_t* packed;  // block 0 of the cache (or tensor)
+    const uint8_t* scales;  // block 0 of the cache (or tensor)
+    const float* amax;      // chunk amax array (or the tensor amax)
+    void* y;                // receives block blk_lo onwards
 };
 
 struct DequantBatch {
     DequantTensor t[kMaxBatch];
-    uint64_t n_blocks;          // blocks per tensor in the range
-    uint64_t block0;            // cache block index of the range's first block
-    uint32_t blocks_per_chunk;  // chunked form only
+    uint64_t blk_lo, blk_hi;    // block range [blk_lo, blk_hi) to dequantize
+    uint64_t blocks_per_chunk;  // blocks sharing one amax
+    uint64_t chunk0;            // chunk of blk_lo; blockIdx.y counts chunks from here
 };
+
+// Work layout. Every CTA owns one contiguous tile of its tensor, and consecutive CTAs
+// own consecutive tiles, so the CTAs resident at any moment stream through one compact
+// window of memory. On B200 this measured 10-15% more DRAM throughput than a
+// persistent grid-stride loop over the same bytes.
+constexpr int kAmaxIters = 4;  // blocks per thread in amax_kernel
 
 // ---------------------------------------------------------------- kernels
 
@@ -85,27 +91,26 @@ __global__ void __launch_bounds__(64) zero_kernel(const ZeroBatch z)
         *z.out[i] = 0u;
 }
 
+// grid (tiles, tensors); a tile is kThreads * kAmaxIters blocks.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxBatch B)
 {
     const char* x = static_cast<const char*>(B.x[blockIdx.y]);
-    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
-    uint64_t b = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const uint64_t base = static_cast<uint64_t>(blockIdx.x) * (kThreads * kAmaxIters) + threadIdx.x;
+    uint32_t w[kAmaxIters][8];
+#pragma unroll
+    for (int i = 0; i < kAmaxIters; ++i) {
+        const uint64_t b = base + i * kThreads;
+        if (b < B.n_blocks)
+            ld_nc_v8(x + b * 32, w[i]);
+        else
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                w[i][k] = 0u;
+    }
     uint32_t m = 0;
-    // four independent 32-byte loads in flight per thread
-    for (; b + 3 * stride < B.n_blocks; b += 4 * stride) {
-        uint32_t w0[8], w1[8], w2[8], w3[8];
-        ld_nc_v8(x + b * 32, w0);
-        ld_nc_v8(x + (b + stride) * 32, w1);
-        ld_nc_v8(x + (b + 2 * stride) * 32, w2);
-        ld_nc_v8(x + (b + 3 * stride) * 32, w3);
-        m = max(m, max(max(block_absmax_bits(w0), block_absmax_bits(w1)),
-                       max(block_absmax_bits(w2), block_absmax_bits(w3))));
-    }
-    for (; b < B.n_blocks; b += stride) {
-        uint32_t w[8];
-        ld_nc_v8(x + b * 32, w);
-        m = max(m, block_absmax_bits(w));
-    }
+#pragma unroll
+    for (int i = 0; i < kAmaxIters; ++i)
+        m = max(m, block_absmax_bits(w[i]));
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     __shared__ uint32_t warp_max[kThreads / 32];
     if ((threadIdx.x & 31) == 0)
@@ -127,136 +132,146 @@ __device__ __forceinline__ float safe_rcp(float S)
     return inv == __int_as_float(0x7F800000) ? 0.0f : inv;
 }
 
-// The e2m1 codes of one block under decoded scale reciprocal `inv` (two words).
-__device__ __forceinline__ void encode_values(const float (&x)[kBlock], float inv, uint32_t& q0, uint32_t& q1)
+// Per-CTA tables of the decoded block scale S(c) = e4m3_value(c) * gs and of its safe
+// reciprocal, for every e4m3 code c the quantizer can produce (0..126).
+struct ScaleTables {
+    float S[128];
+    float inv[128];
+};
+
+__device__ __forceinline__ void build_scale_tables(ScaleTables& t, float gs)
 {
+    for (int c = threadIdx.x; c < 128; c += kThreads) {
+        float v, unused;
+        e4m3x2_to_f32(static_cast<uint32_t>(c), v, unused);
+        const float S = c == 127 ? 0.0f : __fmul_rn(v, gs);
+        t.S[c] = S;
+        t.inv[c] = safe_rcp(S);
+    }
+    __syncthreads();
+}
+
+// The block's 16 bf16 values as eight fp32 pairs (element 2j low, 2j + 1 high).
+__device__ __forceinline__ void block_pairs(const uint32_t (&w)[8], uint64_t (&xp)[8])
+{
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        xp[j] = f32x2_pack(bf16lo_to_f32(w[j]), bf16hi_to_f32(w[j]));
+}
+
+// The e2m1 codes of one block under decoded-scale reciprocal inv (two words).
+__device__ __forceinline__ void encode_values(const uint64_t (&xp)[8], float inv, uint32_t& q0, uint32_t& q1)
+{
+    const uint64_t inv2 = f32x2_pack(inv, inv);
     float v0[8], v1[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        v0[i] = __fmul_rn(x[i], inv);
-        v1[i] = __fmul_rn(x[8 + i], inv);
+    for (int j = 0; j < 4; ++j) {
+        f32x2_unpack(f32x2_mul(xp[j], inv2), v0[2 * j], v0[2 * j + 1]);
+        f32x2_unpack(f32x2_mul(xp[4 + j], inv2), v1[2 * j], v1[2 * j + 1]);
     }
     q0 = e2m1x8_from_f32(v0);
     q1 = e2m1x8_from_f32(v1);
 }
 
 // One mse candidate: the codes of the block under scale S (reciprocal inv) and their
-// squared reconstruction error -- residuals x - value*S by one fma each, squares
-// accumulated by fma into even- and odd-position partial sums, then added.
-__device__ __forceinline__ float encode_values_sq_error(const float (&x)[kBlock], float S, float inv, uint32_t& q0,
+// squared reconstruction error. Residuals x - value*S are one fma each (computed as
+// fma(value, -S, x)); squares accumulate by fma into the pair (even-position sum,
+// odd-position sum) in index order; the two sums are then added.
+__device__ __forceinline__ float encode_values_sq_error(const uint64_t (&xp)[8], float S, float inv, uint32_t& q0,
                                                         uint32_t& q1)
 {
+    const uint64_t inv2 = f32x2_pack(inv, inv);
+    const uint64_t nS2 = f32x2_pack(-S, -S);
     float v0[8], v1[8], val0[8], val1[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        v0[i] = __fmul_rn(x[i], inv);
-        v1[i] = __fmul_rn(x[8 + i], inv);
+    for (int j = 0; j < 4; ++j) {
+        f32x2_unpack(f32x2_mul(xp[j], inv2), v0[2 * j], v0[2 * j + 1]);
+        f32x2_unpack(f32x2_mul(xp[4 + j], inv2), v1[2 * j], v1[2 * j + 1]);
     }
     q0 = e2m1x8_encode_decode(v0, val0);
     q1 = e2m1x8_encode_decode(v1, val1);
-    float se = 0.0f, so = 0.0f;
+    uint64_t acc = f32x2_pack(0.0f, 0.0f);
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-        const float de = __fmaf_rn(-val0[i], S, x[i]);
-        const float dodd = __fmaf_rn(-val0[i + 1], S, x[i + 1]);
-        se = __fmaf_rn(de, de, se);
-        so = __fmaf_rn(dodd, dodd, so);
+    for (int j = 0; j < 4; ++j) {
+        const uint64_t d = f32x2_fma(f32x2_pack(val0[2 * j], val0[2 * j + 1]), nS2, xp[j]);
+        acc = f32x2_fma(d, d, acc);
     }
 #pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-        const float de = __fmaf_rn(-val1[i], S, x[8 + i]);
-        const float dodd = __fmaf_rn(-val1[i + 1], S, x[8 + i + 1]);
-        se = __fmaf_rn(de, de, se);
-        so = __fmaf_rn(dodd, dodd, so);
+    for (int j = 0; j < 4; ++j) {
+        const uint64_t d = f32x2_fma(f32x2_pack(val1[2 * j], val1[2 * j + 1]), nS2, xp[4 + j]);
+        acc = f32x2_fma(d, d, acc);
     }
+    float se, so;
+    f32x2_unpack(acc, se, so);
     return __fadd_rn(se, so);
 }
 
 // Quantize one block held in w (16 bf16). Returns the scale code; q0/q1 get the codes.
 template <int RULE>
-__device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], float gs, bool gs_zero, uint32_t& q0,
-                                                   uint32_t& q1)
+__device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], float gs, bool gs_zero,
+                                                   const ScaleTables& tab, uint32_t& q0, uint32_t& q1)
 {
     const float amax_b = __uint_as_float(block_absmax_bits(w) << 16);
-    float x[kBlock];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        x[2 * j] = bf16lo_to_f32(w[j]);
-        x[2 * j + 1] = bf16hi_to_f32(w[j]);
-    }
+    uint64_t xp[8];
+    block_pairs(w, xp);
     if (RULE == KVQ_RULE_STATIC_6 || RULE == KVQ_RULE_STATIC_4) {
-        const float s = RULE == KVQ_RULE_STATIC_6 ? __fdiv_rn(amax_b, 6.0f) : __fdiv_rn(amax_b, 4.0f);
-        const float r = __fdiv_rn(s, gs);
-        const uint32_t c = gs_zero ? 0u : (e4m3x2_from_f32(0.0f, r) & 0xFFu);
-        float S, unused;
-        e4m3x2_to_f32(c, S, unused);
-        S = __fmul_rn(S, gs);
-        encode_values(x, safe_rcp(S), q0, q1);
+        // amax_b / 4 is exact, so the product by 0.25 equals the IEEE quotient
+        const float s = RULE == KVQ_RULE_STATIC_6 ? __fdiv_rn(amax_b, 6.0f) : __fmul_rn(amax_b, 0.25f);
+        const uint32_t c = gs_zero ? 0u : (e4m3x2_from_f32(0.0f, __fdiv_rn(s, gs)) & 0xFFu);
+        encode_values(xp, tab.inv[c], q0, q1);
         return c;
     } else {
-        const float s6 = __fdiv_rn(amax_b, 6.0f);
-        const float s4 = __fdiv_rn(amax_b, 4.0f);
-        const float r6 = __fdiv_rn(s6, gs);
-        const float r4 = __fdiv_rn(s4, gs);
+        const float r6 = __fdiv_rn(__fdiv_rn(amax_b, 6.0f), gs);
+        const float r4 = __fdiv_rn(__fmul_rn(amax_b, 0.25f), gs);
         const uint32_t c2 = gs_zero ? 0u : e4m3x2_from_f32(r4, r6);  // c6 in bits 0..7, c4 in 8..15
-        float S6, S4;
-        e4m3x2_to_f32(c2, S6, S4);
-        S6 = __fmul_rn(S6, gs);
-        S4 = __fmul_rn(S4, gs);
+        const uint32_t c6 = c2 & 0xFFu, c4 = c2 >> 8;
         uint32_t a0, a1, b0, b1;
-        const float e6 = encode_values_sq_error(x, S6, safe_rcp(S6), a0, a1);
-        const float e4 = encode_values_sq_error(x, S4, safe_rcp(S4), b0, b1);
+        const float e6 = encode_values_sq_error(xp, tab.S[c6], tab.inv[c6], a0, a1);
+        const float e4 = encode_values_sq_error(xp, tab.S[c4], tab.inv[c4], b0, b1);
         const bool use4 = e4 < e6;
         q0 = use4 ? b0 : a0;
         q1 = use4 ? b1 : a1;
-        return use4 ? (c2 >> 8) : (c2 & 0xFFu);
+        return use4 ? c4 : c6;
     }
 }
 
-// BPT = blocks per thread per step (1 or 2). With BPT = 2 the packed pointer must be
-// 16-byte aligned and the scale pointer 2-byte aligned.
+// grid (tiles, tensors), one unit of BPT blocks per thread. The tiles and tensors are
+// walked in the reverse of amax_kernel's order, so the data amax_kernel read last (still
+// in L2) is quantized first. With BPT = 2 the packed pointer must be 16-byte and the
+// scale pointer 2-byte aligned.
 template <int RULE, int BPT>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
 {
-    const QuantTensor& T = B.t[blockIdx.y];
+    __shared__ ScaleTables tab;
+    const QuantTensor& T = B.t[gridDim.y - 1 - blockIdx.y];
     const float amax = __ldg(T.amax);
     const float gs = __fdiv_rn(amax, kGlobalDen);
     const bool gs_zero = gs == 0.0f;
     if (T.amax_copy != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
         *T.amax_copy = amax;
+    build_scale_tables(tab, gs);
 
     const char* x = static_cast<const char*>(T.x);
-    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
-    const uint64_t n_units = B.n_blocks / BPT;
-    for (uint64_t u = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x; u < n_units; u += stride) {
-        if (BPT == 2) {
-            uint32_t w0[8], w1[8];
-            ld_nc_v8(x + u * 64, w0);
-            ld_nc_v8(x + u * 64 + 32, w1);
-            uint32_t q0, q1, q2, q3;
-            const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, q0, q1);
-            const uint32_t c1 = quantize_block<RULE>(w1, gs, gs_zero, q2, q3);
-            st_v4(T.packed + u * 16, q0, q1, q2, q3);
-            *reinterpret_cast<uint16_t*>(T.scales + u * 2) = static_cast<uint16_t>(c0 | (c1 << 8));
-        } else {
-            uint32_t w0[8];
-            ld_nc_v8(x + u * 32, w0);
-            uint32_t q0, q1;
-            const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, q0, q1);
-            st_v2(T.packed + u * 8, q0, q1);
-            T.scales[u] = static_cast<uint8_t>(c0);
-        }
-    }
-    if (BPT == 2) {  // odd block count: the last block alone
-        const uint64_t b = n_units * 2 + static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
-        if (b < B.n_blocks) {
-            uint32_t w0[8];
-            ld_nc_v8(x + b * 32, w0);
-            uint32_t q0, q1;
-            const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, q0, q1);
-            st_v2(T.packed + b * 8, q0, q1);
-            T.scales[b] = static_cast<uint8_t>(c0);
-        }
+    const uint64_t u = static_cast<uint64_t>(gridDim.x - 1 - blockIdx.x) * kThreads + threadIdx.x;
+    const uint64_t b0 = u * BPT;
+    if (b0 >= B.n_blocks)
+        return;
+    if (BPT == 2 && b0 + 1 < B.n_blocks) {
+        uint32_t w0[8], w1[8];
+        ld_nc_v8(x + b0 * 32, w0);
+        ld_nc_v8(x + b0 * 32 + 32, w1);
+        uint32_t q0, q1, q2, q3;
+        const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, tab, q0, q1);
+        const uint32_t c1 = quantize_block<RULE>(w1, gs, gs_zero, tab, q2, q3);
+        st_v4(T.packed + b0 * 8, q0, q1, q2, q3);
+        *reinterpret_cast<uint16_t*>(T.scales + b0) = static_cast<uint16_t>(c0 | (c1 << 8));
+    } else {  // BPT == 1, or the odd last block of a pair unit
+        uint32_t w0[8];
+        ld_nc_v8(x + b0 * 32, w0);
+        uint32_t q0, q1;
+        const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, tab, q0, q1);
+        st_v2(T.packed + b0 * 8, q0, q1);
+        T.scales[b0] = static_cast<uint8_t>(c0);
     }
 }
 
@@ -266,60 +281,60 @@ __device__ __forceinline__ void dequant_block(uint32_t q0, uint32_t q1, uint32_t
     float S, unused;
     e4m3x2_to_f32(c & 0xFFu, S, unused);
     S = __fmul_rn(S, gs);
+    const uint64_t S2 = f32x2_pack(S, S);
     float v[8];
     e2m1x8_to_f32(q0, v);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-        y[j] = bf16x2_from_f32(__fmul_rn(v[2 * j + 1], S), __fmul_rn(v[2 * j], S));
+    for (int j = 0; j < 4; ++j) {
+        float lo, hi;
+        f32x2_unpack(f32x2_mul(f32x2_pack(v[2 * j], v[2 * j + 1]), S2), lo, hi);
+        y[j] = bf16x2_from_f32(hi, lo);
+    }
     e2m1x8_to_f32(q1, v);
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-        y[4 + j] = bf16x2_from_f32(__fmul_rn(v[2 * j + 1], S), __fmul_rn(v[2 * j], S));
+    for (int j = 0; j < 4; ++j) {
+        float lo, hi;
+        f32x2_unpack(f32x2_mul(f32x2_pack(v[2 * j], v[2 * j + 1]), S2), lo, hi);
+        y[4 + j] = bf16x2_from_f32(hi, lo);
+    }
 }
 
-template <bool CHUNKED>
-__device__ __forceinline__ float block_gs(const DequantTensor& T, const DequantBatch& B, uint64_t b, float gs_tensor)
-{
-    if (!CHUNKED)
-        return gs_tensor;
-    const uint32_t chunk = static_cast<uint32_t>((B.block0 + b) / B.blocks_per_chunk);
-    return __fdiv_rn(__ldg(T.amax + chunk), kGlobalDen);
-}
-
-template <int BPT, bool CHUNKED>
+// grid (tiles, chunks, tensors). Each CTA lies inside one chunk, so its amax (and global
+// scale) is one load per CTA. Blocks are numbered from block 0 of the cache; units of BPT
+// blocks are aligned to that numbering, and blocks outside [blk_lo, blk_hi) are skipped.
+template <int BPT>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantBatch B)
 {
-    const DequantTensor& T = B.t[blockIdx.y];
-    const float gs_tensor = CHUNKED ? 0.0f : __fdiv_rn(__ldg(T.amax), kGlobalDen);
+    const DequantTensor& T = B.t[blockIdx.z];
+    const uint64_t chunk = B.chunk0 + blockIdx.y;
+    const uint64_t c_lo = chunk * B.blocks_per_chunk;
+    const uint64_t lo = c_lo > B.blk_lo ? c_lo : B.blk_lo;
+    const uint64_t c_hi = c_lo + B.blocks_per_chunk;
+    const uint64_t hi = c_hi < B.blk_hi ? c_hi : B.blk_hi;
+    if (lo >= hi)
+        return;
+    const uint64_t u = lo / BPT + static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const uint64_t b0 = u * BPT;
+    if (b0 >= hi)
+        return;
+    const float gs = __fdiv_rn(__ldg(T.amax + chunk), kGlobalDen);
     char* y = static_cast<char*>(T.y);
-    const uint64_t stride = static_cast<uint64_t>(gridDim.x) * kThreads;
-    const uint64_t n_units = B.n_blocks / BPT;
-    for (uint64_t u = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x; u < n_units; u += stride) {
-        if (BPT == 2) {
-            const uint4 q = ld_nc_v4(T.packed + u * 16);
-            const uint32_t c = __ldg(reinterpret_cast<const uint16_t*>(T.scales) + u);
-            uint32_t y0[8], y1[8];
-            dequant_block(q.x, q.y, c, block_gs<CHUNKED>(T, B, 2 * u, gs_tensor), y0);
-            dequant_block(q.z, q.w, c >> 8, block_gs<CHUNKED>(T, B, 2 * u + 1, gs_tensor), y1);
-            st_v8(y + u * 64, y0);
-            st_v8(y + u * 64 + 32, y1);
-        } else {
-            const uint2 q = ld_nc_v2(T.packed + u * 8);
-            const uint32_t c = __ldg(T.scales + u);
-            uint32_t y0[8];
-            dequant_block(q.x, q.y, c, block_gs<CHUNKED>(T, B, u, gs_tensor), y0);
-            st_v8(y + u * 32, y0);
+    if (BPT == 2 && b0 + 1 < hi) {  // both blocks of the unit readable (block b0 may be lo - 1)
+        const uint4 q = ld_nc_v4(T.packed + b0 * 8);
+        const uint32_t c = __ldg(reinterpret_cast<const uint16_t*>(T.scales + b0));
+        uint32_t y0[8];
+        if (b0 >= lo) {
+            dequant_block(q.x, q.y, c, gs, y0);
+            st_v8(y + (b0 - B.blk_lo) * 32, y0);
         }
-    }
-    if (BPT == 2) {
-        const uint64_t b = n_units * 2 + static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
-        if (b < B.n_blocks) {
-            const uint2 q = ld_nc_v2(T.packed + b * 8);
-            const uint32_t c = __ldg(T.scales + b);
-            uint32_t y0[8];
-            dequant_block(q.x, q.y, c, block_gs<CHUNKED>(T, B, b, gs_tensor), y0);
-            st_v8(y + b * 32, y0);
-        }
+        dequant_block(q.z, q.w, c >> 8, gs, y0);
+        st_v8(y + (b0 + 1 - B.blk_lo) * 32, y0);
+    } else {  // BPT == 1, or a unit whose second block is past the range
+        const uint64_t b = (BPT == 2 && b0 < lo) ? b0 + 1 : b0;
+        const uint2 q = ld_nc_v2(T.packed + b * 8);
+        uint32_t y0[8];
+        dequant_block(q.x, q.y, __ldg(T.scales + b), gs, y0);
+        st_v8(y + (b - B.blk_lo) * 32, y0);
     }
 }
 
@@ -353,24 +368,11 @@ kvq_status check_launch(const char* what)
     return KVQ_OK;
 }
 
-// CTAs per tensor for a grid-stride kernel: enough to fill every SM at the kernel's
-// occupancy, spread over the tensors of the batch, and no more than the work needs.
-template <typename K>
-kvq_status grid_x(K kernel, uint64_t units_per_tensor, int n_tensors, unsigned* gx)
+// CTAs along x for `units` units of one tensor, kThreads (times `per_thread`) per CTA.
+unsigned tiles(uint64_t units, uint64_t per_thread = 1)
 {
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess) {
-        cudaError_t e = cudaGetLastError();
-        return fail(KVQ_ERR_CUDA, "device query: %s", cudaGetErrorString(e));
-    }
-    uint64_t full = static_cast<uint64_t>(sms) * static_cast<uint64_t>(per_sm > 0 ? per_sm : 1);
-    uint64_t want = (full + n_tensors - 1) / n_tensors;
-    uint64_t need = (units_per_tensor + kThreads - 1) / kThreads;
-    uint64_t g = want < need ? want : need;
-    *gx = static_cast<unsigned>(g < 1 ? 1 : g);
-    return KVQ_OK;
+    const uint64_t per_cta = static_cast<uint64_t>(kThreads) * per_thread;
+    return static_cast<unsigned>((units + per_cta - 1) / per_cta);
 }
 
 kvq_status check_rule(kvq_scale_rule rule)
@@ -400,6 +402,7 @@ kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scal
 {
     if (n == 0 || qb.n_blocks == 0)
         return KVQ_OK;
+    kvq_status st;
     if (compute_amax) {
         ZeroBatch z{};
         AmaxBatch ab{};
@@ -411,76 +414,61 @@ kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scal
         z.n = n;
         ab.n_blocks = qb.n_blocks;
         zero_kernel<<<1, 64, 0, s>>>(z);
-        kvq_status st = check_launch("zero_kernel");
-        if (st != KVQ_OK)
+        if ((st = check_launch("zero_kernel")) != KVQ_OK)
             return st;
-        unsigned gx;
-        if ((st = grid_x(amax_kernel, qb.n_blocks, n, &gx)) != KVQ_OK)
-            return st;
-        amax_kernel<<<dim3(gx, n), kThreads, 0, s>>>(ab);
+        amax_kernel<<<dim3(tiles(qb.n_blocks, kAmaxIters), n), kThreads, 0, s>>>(ab);
         if ((st = check_launch("amax_kernel")) != KVQ_OK)
             return st;
     }
-    bool pairs = qb.n_blocks >= 2;
+    bool pairs = true;
     for (int i = 0; i < n; ++i)
         pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
-    const uint64_t units = pairs ? qb.n_blocks / 2 : qb.n_blocks;
-    unsigned gx;
-    kvq_status st;
-#define KVQ_LAUNCH_Q(R, BPT)                                                        \
-    do {                                                                            \
-        if ((st = grid_x(quantize_kernel<R, BPT>, units, n, &gx)) != KVQ_OK)        \
-            return st;                                                              \
-        quantize_kernel<R, BPT><<<dim3(gx, n), kThreads, 0, s>>>(qb);               \
-    } while (0)
+    const dim3 grid(tiles(pairs ? (qb.n_blocks + 1) / 2 : qb.n_blocks), n);
     if (pairs) {
         if (rule == KVQ_RULE_STATIC_6)
-            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_6, 2);
+            quantize_kernel<KVQ_RULE_STATIC_6, 2><<<grid, kThreads, 0, s>>>(qb);
         else if (rule == KVQ_RULE_STATIC_4)
-            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_4, 2);
+            quantize_kernel<KVQ_RULE_STATIC_4, 2><<<grid, kThreads, 0, s>>>(qb);
         else
-            KVQ_LAUNCH_Q(KVQ_RULE_MSE, 2);
+            quantize_kernel<KVQ_RULE_MSE, 2><<<grid, kThreads, 0, s>>>(qb);
     } else {
         if (rule == KVQ_RULE_STATIC_6)
-            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_6, 1);
+            quantize_kernel<KVQ_RULE_STATIC_6, 1><<<grid, kThreads, 0, s>>>(qb);
         else if (rule == KVQ_RULE_STATIC_4)
-            KVQ_LAUNCH_Q(KVQ_RULE_STATIC_4, 1);
+            quantize_kernel<KVQ_RULE_STATIC_4, 1><<<grid, kThreads, 0, s>>>(qb);
         else
-            KVQ_LAUNCH_Q(KVQ_RULE_MSE, 1);
+            quantize_kernel<KVQ_RULE_MSE, 1><<<grid, kThreads, 0, s>>>(qb);
     }
-#undef KVQ_LAUNCH_Q
     return check_launch("quantize_kernel");
 }
 
-kvq_status run_dequantize(const DequantBatch& db, int n, bool chunked, cudaStream_t s)
+// Dequantize blocks [blk_lo, blk_hi) of n equally laid-out tensors; packed/scales point at
+// block 0 of each. One launch per group of at most 65535 chunks (the grid's y limit).
+kvq_status run_dequantize(DequantBatch db, int n, cudaStream_t s)
 {
-    if (n == 0 || db.n_blocks == 0)
+    if (n == 0 || db.blk_hi <= db.blk_lo)
         return KVQ_OK;
-    bool pairs = db.n_blocks >= 2;
+    bool pairs = true;
     for (int i = 0; i < n; ++i)
         pairs = pairs && aligned(db.t[i].packed, 16) && aligned(db.t[i].scales, 2);
-    const uint64_t units = pairs ? db.n_blocks / 2 : db.n_blocks;
-    unsigned gx;
-    kvq_status st;
-#define KVQ_LAUNCH_D(BPT, CH)                                                     \
-    do {                                                                          \
-        if ((st = grid_x(dequant_kernel<BPT, CH>, units, n, &gx)) != KVQ_OK)      \
-            return st;                                                            \
-        dequant_kernel<BPT, CH><<<dim3(gx, n), kThreads, 0, s>>>(db);             \
-    } while (0)
-    if (pairs) {
-        if (chunked)
-            KVQ_LAUNCH_D(2, true);
+    const int bpt = pairs ? 2 : 1;
+    const uint64_t bpc = db.blocks_per_chunk;
+    const uint64_t first = db.blk_lo / bpc, last = (db.blk_hi - 1) / bpc;
+    // units of one chunk, plus one for a chunk that starts inside a unit
+    const unsigned gx = tiles((bpc + bpt - 1) / bpt + 1);
+    for (uint64_t c0 = first; c0 <= last; c0 += 65535) {
+        const uint64_t nc = (last - c0 + 1) < 65535 ? (last - c0 + 1) : 65535;
+        db.chunk0 = c0;
+        const dim3 grid(gx, static_cast<unsigned>(nc), n);
+        if (pairs)
+            dequant_kernel<2><<<grid, kThreads, 0, s>>>(db);
         else
-            KVQ_LAUNCH_D(2, false);
-    } else {
-        if (chunked)
-            KVQ_LAUNCH_D(1, true);
-        else
-            KVQ_LAUNCH_D(1, false);
+            dequant_kernel<1><<<grid, kThreads, 0, s>>>(db);
+        kvq_status st = check_launch("dequant_kernel");
+        if (st != KVQ_OK)
+            return st;
     }
-#undef KVQ_LAUNCH_D
-    return check_launch("dequant_kernel");
+    return KVQ_OK;
 }
 
 kvq_status check_cache(const kvq_cache* c, const char* what)
@@ -559,12 +547,14 @@ kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const fl
     if (!aligned(y, 32) || !aligned(packed, 8) || !aligned(amax, 4))
         return fail(KVQ_ERR_MISALIGNED, "kvq_dequantize: y must be 32-byte, packed 8-byte, amax 4-byte aligned");
     DequantBatch db{};
-    db.n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
+    db.blk_lo = 0;
+    db.blk_hi = static_cast<uint64_t>(n_elems) / kBlock;
+    db.blocks_per_chunk = db.blk_hi;  // one chunk: the tensor
     db.t[0].packed = packed;
     db.t[0].scales = scales;
     db.t[0].amax = amax;
     db.t[0].y = y;
-    if ((st = run_dequantize(db, 1, false, reinterpret_cast<cudaStream_t>(stream))) != KVQ_OK)
+    if ((st = run_dequantize(db, 1, reinterpret_cast<cudaStream_t>(stream))) != KVQ_OK)
         return st;
     return ok();
 }
@@ -670,17 +660,17 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
     for (int base = 0; base < n_tensors; base += kMaxBatch) {
         const int n = n_tensors - base < kMaxBatch ? n_tensors - base : kMaxBatch;
         DequantBatch db{};
-        db.n_blocks = static_cast<uint64_t>(row_end - row_begin) * bpr;
-        db.block0 = static_cast<uint64_t>(row_begin) * bpr;
-        db.blocks_per_chunk = static_cast<uint32_t>(static_cast<uint64_t>(rpc) * bpr);
+        db.blk_lo = static_cast<uint64_t>(row_begin) * bpr;
+        db.blk_hi = static_cast<uint64_t>(row_end) * bpr;
+        db.blocks_per_chunk = static_cast<uint64_t>(rpc) * bpr;
         for (int i = 0; i < n; ++i) {
             const kvq_cache* c = &caches[base + i];
-            db.t[i].packed = c->packed + db.block0 * 8;
-            db.t[i].scales = c->scales + db.block0;
+            db.t[i].packed = c->packed;
+            db.t[i].scales = c->scales;
             db.t[i].amax = c->amax;
             db.t[i].y = ys[base + i];
         }
-        if ((st = run_dequantize(db, n, true, s)) != KVQ_OK)
+        if ((st = run_dequantize(db, n, s)) != KVQ_OK)
             return st;
     }
     return ok();

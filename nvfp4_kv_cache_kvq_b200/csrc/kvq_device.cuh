@@ -51,11 +51,12 @@ __device__ __forceinline__ void st_v4(void* p, uint32_t a, uint32_t b, uint32_t 
     asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Per-16-bit-lane unsigned max of two words.
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
+// Lane-wise max(|a|, |b|) of two bf16x2 words (the sign bit of each lane is the xor of
+// the operands' signs and is cleared by the caller).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
 {
     uint32_t d;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
 
@@ -63,13 +64,39 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
 // finite values the integer order of |bf16| bit patterns is their numeric order.
 __device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&w)[8])
 {
-    constexpr uint32_t kAbs = 0x7FFF7FFFu;
-    uint32_t m01 = max_u16x2(w[0] & kAbs, w[1] & kAbs);
-    uint32_t m23 = max_u16x2(w[2] & kAbs, w[3] & kAbs);
-    uint32_t m45 = max_u16x2(w[4] & kAbs, w[5] & kAbs);
-    uint32_t m67 = max_u16x2(w[6] & kAbs, w[7] & kAbs);
-    uint32_t m = max_u16x2(max_u16x2(m01, m23), max_u16x2(m45, m67));
+    const uint32_t m = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3])),
+                                     absmax_bf16x2(absmax_bf16x2(w[4], w[5]), absmax_bf16x2(w[6], w[7])))
+                       & 0x7FFF7FFFu;
     return max(m & 0xFFFFu, m >> 16);
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): the low 32 bits hold the first value.
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi)
+{
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+
+__device__ __forceinline__ void f32x2_unpack(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// Lane-wise a * b, rounded to nearest even.
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Lane-wise fused a * b + c, one rounding to nearest even.
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }

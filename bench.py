@@ -46,6 +46,30 @@ B_DEQUANT = 2.5625  # 0.5625 B read + bf16 written, per element
 L2_BYTES = 126 * 2 ** 20
 
 
+def kernel_source_sha256() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for rel in ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kind: str):
+    """DRAM bytes per element of a kernel kind from the committed ncu summary
+    (profiles/traffic.json), or None when the kernels changed since that capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("source_sha256") != kernel_source_sha256():
+        return None
+    k = t.get("kernels", {}).get(kind)
+    return None if k is None else float(k["dram_bytes_per_elem"])
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -388,20 +412,29 @@ WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep)}
 
 # ---------------------------------------------------------------------------- runner
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE). The process
+    group only carries the barrier around the timed region and the max of the step
+    times: the workload itself has no exchange (every rank is an independent replica)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend == "nccl":
+        torch.cuda.set_device(local if world > 1 else 0)
     if world > 1:
         import datetime
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
+
+
+def _reduce_device():
+    import torch.distributed as dist
+
+    return torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
 
 
 def barrier(world):
@@ -416,9 +449,15 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch.distributed as dist
 
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=_reduce_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_gbs(world: int, bytes_per_rank_step: float, max_ms_per_step: float) -> float:
+    """Whole-job GB/s: every rank processed bytes_per_rank_step per step; the step time
+    is the slowest rank's."""
+    return world * bytes_per_rank_step / (max_ms_per_step * 1e-3) / 1e9
 
 
 def cpu_baseline(wl, budget_s):
@@ -557,17 +596,21 @@ def main():
     mean_ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
 
     bytes_step = sum(s.bytes_alg for s in segs)
-    value = world * bytes_step / (mean_ms * 1e-3) / 1e9
+    value = aggregate_gbs(world, bytes_step, mean_ms)
     peak, peak_src = peaks()
     kind_bytes = {k: sum(s.bytes_alg for s in segs if s.kind == k) for k in kinds}
     kind_launch = {k: sum(s.launches for s in segs if s.kind == k) for k in kinds}
     dom = max(kinds, key=lambda k: kind_ms[k])
     dom_ms = kind_ms[dom] / args.steps
     achieved = kind_bytes[dom] / (dom_ms * 1e-3) / 1e9
+    per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT}[dom]
+    tb = measured_traffic(dom)
+    elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                "traffic": None, "launches_per_step": kind_launch[dom],
-                "alg_bytes_per_step": kind_bytes[dom], "ms_per_step": dom_ms}
+                "traffic": None if tb is None else tb * elems_per_launch,
+                "alg_bytes_per_launch": kind_bytes[dom] / kind_launch[dom],
+                "launches_per_step": kind_launch[dom], "ms_per_step": dom_ms}
     per_kind = {k: {"ms_per_step": kind_ms[k] / args.steps,
                     "GB_s": kind_bytes[k] / (kind_ms[k] / args.steps * 1e-3) / 1e9 if kind_ms[k] else None,
                     "launches_per_step": kind_launch[k]} for k in kinds}
@@ -622,7 +665,7 @@ def run_e2e(args, wl, segs, bytes_step, world):
         torch.cuda.synchronize()
         ms.append(events[0].elapsed_time(events[-1]))
     mean_ms = max_over_ranks(sum(ms) / len(ms), world)
-    return {"value": world * bytes_step / (mean_ms * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": mean_ms,
+    return {"value": aggregate_gbs(world, bytes_step, mean_ms), "unit": "GB/s", "ms_per_step": mean_ms,
             "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes, "steps": steps}
 
 

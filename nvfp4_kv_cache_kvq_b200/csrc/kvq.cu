@@ -206,23 +206,62 @@ __device__ __forceinline__ float encode_values_sq_error(const uint64_t (&xp)[8],
     return __fadd_rn(se, so);
 }
 
+// Correctly rounded quotients without a division per block: Markstein's correction step
+// (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990). With y = RN(1/b) (CUDA's IEEE reciprocal,
+// __frcp_rn) and q = RN(a*y), the remainder r = a - b*q is exact as one fma and
+// RN(q + r*y) is the IEEE quotient RN(a/b), as long as nothing under- or overflows.
+// For a/6 this holds for every bf16 amax (checked exhaustively). For s/gs it holds when
+// gs is in [2^-80, 2^125] and the quotient is in [2^-12, 464], the only range where the
+// quotient decides an e4m3 code (below 2^-12 every code is 0, above 464 every code
+// saturates to 448). Clamping at 512 keeps an overflowing quotient (a caller's amax_in
+// far below the data) on the saturating side, as the IEEE quotient is.
+struct Quotients {
+    float gs, inv_gs;
+    bool markstein;  // gs in [2^-80, 2^125]; else IEEE division
+};
+
+__device__ __forceinline__ float markstein(float a, float b, float y)
+{
+    const float q = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-q, b, a);
+    return __fmaf_rn(r, y, q);
+}
+
+__device__ __forceinline__ float div6(float a)
+{
+    return markstein(a, 6.0f, __int_as_float(0x3E2AAAAB));  // RN(1/6)
+}
+
+// e4m3 input of a block scale s: (s / gs), exactly where it decides the code. MARK is
+// the per-tensor choice between the corrected product and IEEE division; it is a
+// template parameter so that each kernel path holds only one of the two.
+template <bool MARK>
+__device__ __forceinline__ float scale_ratio(float s, const Quotients& qt)
+{
+    return MARK ? fminf(markstein(s, qt.gs, qt.inv_gs), 512.0f) : __fdiv_rn(s, qt.gs);
+}
+
 // Quantize one block held in w (16 bf16). Returns the scale code; q0/q1 get the codes.
-template <int RULE>
-__device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], float gs, bool gs_zero,
+// With MARK, gs >= 2^-80 is non-zero; otherwise gs == 0 (an all-zero tensor or amax_in
+// == 0) forces every scale code to 0.
+template <int RULE, bool MARK>
+__device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], const Quotients& qt,
                                                    const ScaleTables& tab, uint32_t& q0, uint32_t& q1)
 {
+    const bool gs_zero = !MARK && qt.gs == 0.0f;
     const float amax_b = __uint_as_float(block_absmax_bits(w) << 16);
     uint64_t xp[8];
     block_pairs(w, xp);
     if (RULE == KVQ_RULE_STATIC_6 || RULE == KVQ_RULE_STATIC_4) {
         // amax_b / 4 is exact, so the product by 0.25 equals the IEEE quotient
-        const float s = RULE == KVQ_RULE_STATIC_6 ? __fdiv_rn(amax_b, 6.0f) : __fmul_rn(amax_b, 0.25f);
-        const uint32_t c = gs_zero ? 0u : (e4m3x2_from_f32(0.0f, __fdiv_rn(s, gs)) & 0xFFu);
+        const float s = RULE == KVQ_RULE_STATIC_6 ? div6(amax_b) : __fmul_rn(amax_b, 0.25f);
+        const uint32_t c = gs_zero ? 0u : (e4m3x2_from_f32(0.0f, scale_ratio<MARK>(s, qt)) & 0xFFu);
         encode_values(xp, tab.inv[c], q0, q1);
         return c;
     } else {
-        const float r6 = __fdiv_rn(__fdiv_rn(amax_b, 6.0f), gs);
-        const float r4 = __fdiv_rn(__fmul_rn(amax_b, 0.25f), gs);
+        const float r6 = scale_ratio<MARK>(div6(amax_b), qt);
+        const float r4 = scale_ratio<MARK>(__fmul_rn(amax_b, 0.25f), qt);
         const uint32_t c2 = gs_zero ? 0u : e4m3x2_from_f32(r4, r6);  // c6 in bits 0..7, c4 in 8..15
         const uint32_t c6 = c2 & 0xFFu, c4 = c2 >> 8;
         uint32_t a0, a1, b0, b1;
@@ -232,6 +271,32 @@ __device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], float
         q0 = use4 ? b0 : a0;
         q1 = use4 ? b1 : a1;
         return use4 ? c4 : c6;
+    }
+}
+
+// Unit u of a tensor: blocks [u*BPT, u*BPT + BPT) clipped to n_blocks.
+template <int RULE, int BPT, bool MARK>
+__device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, uint64_t n_blocks,
+                                              const Quotients& qt, const ScaleTables& tab)
+{
+    const char* x = static_cast<const char*>(T.x);
+    const uint64_t b0 = u * BPT;
+    if (BPT == 2 && b0 + 1 < n_blocks) {
+        uint32_t w0[8], w1[8];
+        ld_nc_v8(x + b0 * 32, w0);
+        ld_nc_v8(x + b0 * 32 + 32, w1);
+        uint32_t q0, q1, q2, q3;
+        const uint32_t c0 = quantize_block<RULE, MARK>(w0, qt, tab, q0, q1);
+        const uint32_t c1 = quantize_block<RULE, MARK>(w1, qt, tab, q2, q3);
+        st_v4(T.packed + b0 * 8, q0, q1, q2, q3);
+        *reinterpret_cast<uint16_t*>(T.scales + b0) = static_cast<uint16_t>(c0 | (c1 << 8));
+    } else {  // BPT == 1, or the odd last block of a pair unit
+        uint32_t w0[8];
+        ld_nc_v8(x + b0 * 32, w0);
+        uint32_t q0, q1;
+        const uint32_t c0 = quantize_block<RULE, MARK>(w0, qt, tab, q0, q1);
+        st_v2(T.packed + b0 * 8, q0, q1);
+        T.scales[b0] = static_cast<uint8_t>(c0);
     }
 }
 
@@ -245,34 +310,21 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
     __shared__ ScaleTables tab;
     const QuantTensor& T = B.t[gridDim.y - 1 - blockIdx.y];
     const float amax = __ldg(T.amax);
-    const float gs = __fdiv_rn(amax, kGlobalDen);
-    const bool gs_zero = gs == 0.0f;
+    Quotients qt;
+    qt.gs = __fdiv_rn(amax, kGlobalDen);
+    qt.markstein = qt.gs >= 0x1p-80f && qt.gs <= 0x1p125f;
+    qt.inv_gs = qt.markstein ? __frcp_rn(qt.gs) : 0.0f;
     if (T.amax_copy != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
         *T.amax_copy = amax;
-    build_scale_tables(tab, gs);
+    build_scale_tables(tab, qt.gs);
 
-    const char* x = static_cast<const char*>(T.x);
     const uint64_t u = static_cast<uint64_t>(gridDim.x - 1 - blockIdx.x) * kThreads + threadIdx.x;
-    const uint64_t b0 = u * BPT;
-    if (b0 >= B.n_blocks)
+    if (u * BPT >= B.n_blocks)
         return;
-    if (BPT == 2 && b0 + 1 < B.n_blocks) {
-        uint32_t w0[8], w1[8];
-        ld_nc_v8(x + b0 * 32, w0);
-        ld_nc_v8(x + b0 * 32 + 32, w1);
-        uint32_t q0, q1, q2, q3;
-        const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, tab, q0, q1);
-        const uint32_t c1 = quantize_block<RULE>(w1, gs, gs_zero, tab, q2, q3);
-        st_v4(T.packed + b0 * 8, q0, q1, q2, q3);
-        *reinterpret_cast<uint16_t*>(T.scales + b0) = static_cast<uint16_t>(c0 | (c1 << 8));
-    } else {  // BPT == 1, or the odd last block of a pair unit
-        uint32_t w0[8];
-        ld_nc_v8(x + b0 * 32, w0);
-        uint32_t q0, q1;
-        const uint32_t c0 = quantize_block<RULE>(w0, gs, gs_zero, tab, q0, q1);
-        st_v2(T.packed + b0 * 8, q0, q1);
-        T.scales[b0] = static_cast<uint8_t>(c0);
-    }
+    if (qt.markstein)
+        quantize_unit<RULE, BPT, true>(T, u, B.n_blocks, qt, tab);
+    else
+        quantize_unit<RULE, BPT, false>(T, u, B.n_blocks, qt, tab);
 }
 
 // One block: 8 code bytes (two words) and its scale -> 16 bf16 (eight words).

@@ -91,6 +91,43 @@ def test_e4m3_scale_rounding_of_every_bf16_amax(orc, rule):
     check_full(orc, _bf16(x), rule, 16)
 
 
+def _ulp_step(v, d):
+    """v moved by d fp32 ulps."""
+    v = np.float32(v)
+    for _ in range(abs(d)):
+        v = np.nextafter(v, np.float32(np.inf) if d > 0 else np.float32(0))
+    return float(v)
+
+
+@pytest.mark.parametrize("rule", ["static_6", "static_4", "mse"])
+def test_scale_quotients_at_e4m3_midpoints(orc, rule):
+    """The scale code is e4m3((amax_b / R) / gs): pick amax_in (hence gs) so that the
+    quotient lands on, or a few ulps around, e4m3 rounding midpoints. The code then
+    hinges on the correctly rounded quotient, which the kernel computes without a
+    division (a corrected reciprocal product); the oracle divides."""
+    R = 4.0 if rule == "static_4" else 6.0
+    mags = np.array([orc.e4m3_decode(c) for c in range(127)])
+    mids = (mags[:-1] + mags[1:]) / 2
+    rng = np.random.default_rng(21)
+    a_vals = np.float32([1.0, 0.75, 3.0, 0.5625, 11.0, 1.9375])
+    n_checked = 0
+    for k in range(0, 126, 3):
+        a = float(a_vals[k % a_vals.size])
+        s32 = np.float32(a) / np.float32(R) if R == 6.0 else np.float32(a) * np.float32(0.25)
+        target = np.float32(float(s32) / mids[k] * 2688.0)
+        for d in (-2, -1, 0, 1, 2):
+            amax_in = _ulp_step(target, d)
+            blk = np.concatenate([[a], rng.uniform(-a, a, 15)])
+            x = torch.from_numpy(np.concatenate([blk, rng.standard_normal(16 * 7) * a / 3])).to(torch.bfloat16)
+            p, sc, _ = kvq.kvq_quantize(x.cuda(), 16, rule, amax_in=torch.tensor([amax_in], device="cuda"))
+            torch.cuda.synchronize()
+            pe, se, _ = orc.quantize(bits(x), 16, rule, amax_in=amax_in)
+            assert_same(sc.cpu().numpy(), se, f"scales at midpoint {k} d={d}")
+            assert_same(p.cpu().numpy(), pe, f"packed at midpoint {k} d={d}")
+            n_checked += 1
+    assert n_checked == 42 * 5
+
+
 def test_empty_tensor():
     x = torch.empty(0, dtype=torch.bfloat16, device="cuda")
     amax = torch.full((1,), 5.0, device="cuda")

@@ -12,7 +12,8 @@ sizing, per-chunk amax, block scales, e2m1 packing, and dequantization.
 
 Other workloads: ``single`` ([4096,128], static_6), ``layer`` (one layer's K and V of
 [1,24,4680,128], mse), ``cache`` (30 layers x {K,V} of [1,24,32760,128]; quantize all,
-dequantize per layer), ``sweep`` ([T,128], --tokens).
+dequantize per layer), ``sweep`` ([T,128], --tokens), ``roundtrip`` ([T,128] through the
+fused quantize + dequantize kernel).
 
 Timing: each bench step is captured as CUDA graphs (one per segment: an append, a
 layer loop of reads, ...), replayed with CUDA events between segments on the launching
@@ -407,7 +408,28 @@ class Sweep(Layer):
         return nbytes, time.perf_counter() - t0, f"first {m} of {self.tokens} rows, {reps} repetitions"
 
 
-WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep)}
+class RoundTrip(Sweep):
+    """The fused round trip (quantize + bf16 reconstruction in one pass) on [T, 128]."""
+    name = "roundtrip"
+
+    def __init__(self, args, rank):
+        Sweep.__init__(self, args, rank)
+        self.config["workload"] = (f"fused quantize+dequantize (one pass, codes and bf16 written): "
+                                   f"[{self.tokens},128] N(0,1), rule {self.rule}")
+
+    def segments(self):
+        kvq = self.kvq
+
+        def rt():
+            kvq.kvq_quantize_dequantize(self.x[0], self.D, self.rule, amax_out=self.a[0], packed=self.p[0],
+                                        scales=self.s[0], y=self.y[0])
+        return [Segment("roundtrip", rt, 3, self.n * (B_AMAX + B_QUANT + 2.0), h2d=(self.x[0],))]
+
+    def d2h(self):
+        return [self.p[0], self.s[0], self.a[0], self.y[0]]
+
+
+WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip)}
 
 
 # ---------------------------------------------------------------------------- runner
@@ -603,7 +625,8 @@ def main():
     dom = max(kinds, key=lambda k: kind_ms[k])
     dom_ms = kind_ms[dom] / args.steps
     achieved = kind_bytes[dom] / (dom_ms * 1e-3) / 1e9
-    per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT}[dom]
+    per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
+                "roundtrip": B_AMAX + B_QUANT + 2.0}[dom]
     tb = measured_traffic(dom)
     elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",

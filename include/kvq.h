@@ -112,6 +112,40 @@ kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const fl
                           int32_t head_dim, void* y, kvq_stream_t stream);
 
 /*
+ * kvq_quantize_batch -- n_tensors independent kvq_quantize calls on tensors of the same
+ *   n_elems and head_dim, in one set of launches (e.g. one layer's K and V). Each tensor
+ *   has its own amax, exactly as if quantized alone.
+ *   xs, packed, scales  host arrays of n_tensors device pointers (as in kvq_quantize).
+ *   amax_in   host array of n_tensors device pointers, or NULL: compute every amax.
+ *   amax_out  host array of n_tensors device pointers, or NULL when amax_in is given.
+ *   At most KVQ_MAX_BATCH tensors share a launch; more are split.
+ */
+kvq_status kvq_quantize_batch(const void* const* xs, int32_t n_tensors, int64_t n_elems, int32_t head_dim,
+                              kvq_scale_rule rule, const float* const* amax_in, float* const* amax_out,
+                              uint8_t* const* packed, uint8_t* const* scales, kvq_stream_t stream);
+
+/*
+ * kvq_dequantize_batch -- n_tensors independent kvq_dequantize calls of the same size in
+ *   one set of launches. packed, scales, amax, ys: host arrays of n_tensors device pointers.
+ */
+kvq_status kvq_dequantize_batch(const uint8_t* const* packed, const uint8_t* const* scales,
+                                const float* const* amax, int32_t n_tensors, int64_t n_elems, int32_t head_dim,
+                                void* const* ys, kvq_stream_t stream);
+
+/*
+ * kvq_quantize_dequantize -- the fused round trip ("fake quantization", the
+ *   static_blockwise_fp4_fake_quant of "How NVFP4 Quantization Works in LongLive 2.0",
+ *   "Stage 1"): quantize x and write its bf16 reconstruction y in the same pass. y is
+ *   bit-equal to kvq_quantize followed by kvq_dequantize.
+ *   packed, scales  device outputs as in kvq_quantize, or both NULL to write only y.
+ *   y               device, bf16[n_elems], 32-byte aligned. Written.
+ *   Other arguments as in kvq_quantize.
+ */
+kvq_status kvq_quantize_dequantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
+                                   const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
+                                   void* y, kvq_stream_t stream);
+
+/*
  * A packed K or V cache of one layer, in device memory, token-major: row
  * t * heads + h holds head h of token t, head_dim elements. Rows are grouped in chunks
  * of rows_per_chunk (one chunk = the rows one append writes, e.g. one latent frame of

@@ -52,6 +52,11 @@ def load() -> ctypes.CDLL:
     CP = ctypes.POINTER(_Cache)
     sig = {
         "kvq_quantize": [P, I64, I32, I32, P, P, P, P, P],
+        "kvq_quantize_batch": [ctypes.POINTER(P), I32, I64, I32, I32, ctypes.POINTER(P), ctypes.POINTER(P),
+                               ctypes.POINTER(P), ctypes.POINTER(P), P],
+        "kvq_dequantize_batch": [ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P), I32, I64, I32,
+                                 ctypes.POINTER(P), P],
+        "kvq_quantize_dequantize": [P, I64, I32, I32, P, P, P, P, P, P],
         "kvq_dequantize": [P, P, P, I64, I32, P, P],
         "kvq_append": [CP, I64, P, I64, I32, P],
         "kvq_append_batch": [CP, ctypes.POINTER(I64), ctypes.POINTER(P), I32, I64, I32, P],
@@ -134,6 +139,75 @@ def kvq_dequantize(packed: torch.Tensor, scales: torch.Tensor, amax: torch.Tenso
     _check(load().kvq_dequantize(_dev(packed, "packed"), _dev(scales, "scales"), _dev(amax, "amax"), n,
                                  int(head_dim), _dev(y, "y"), _stream(stream, dev)))
     return y
+
+
+def _ptrs(ts, what):
+    return (ctypes.c_void_p * len(ts))(*[_dev(t, what) for t in ts])
+
+
+def kvq_quantize_batch(xs, head_dim: int | None = None, rule="static_6", amax_in=None, amax_out=None,
+                       packed=None, scales=None, stream=None):
+    """Quantize equally sized bf16 tensors in one set of launches, each with its own amax.
+    Returns (packed list, scales list, amax list)."""
+    n = len(xs)
+    if n == 0:
+        return [], [], []
+    if any(x.dtype != torch.bfloat16 or x.numel() != xs[0].numel() for x in xs):
+        raise ValueError("xs must be bfloat16 tensors of one size")
+    numel = xs[0].numel()
+    head_dim = int(head_dim or xs[0].shape[-1])
+    dev = xs[0].device
+    packed = packed or [torch.empty(numel // 2, dtype=torch.uint8, device=dev) for _ in xs]
+    scales = scales or [torch.empty(numel // BLOCK, dtype=torch.uint8, device=dev) for _ in xs]
+    if amax_in is None and amax_out is None:
+        amax_out = [torch.empty(1, dtype=torch.float32, device=dev) for _ in xs]
+    _check(load().kvq_quantize_batch(_ptrs(xs, "x"), n, numel, head_dim, _rule(rule),
+                                     None if amax_in is None else _ptrs(amax_in, "amax_in"),
+                                     None if amax_out is None else _ptrs(amax_out, "amax_out"),
+                                     _ptrs(packed, "packed"), _ptrs(scales, "scales"), _stream(stream, dev)))
+    return packed, scales, (amax_out if amax_out is not None else amax_in)
+
+
+def kvq_dequantize_batch(packed, scales, amax, head_dim: int, ys=None, stream=None):
+    """Dequantize equally sized tensors in one set of launches. Returns the bf16 list."""
+    n = len(packed)
+    if n == 0:
+        return []
+    numel = packed[0].numel() * 2
+    dev = packed[0].device
+    ys = ys or [torch.empty(numel, dtype=torch.bfloat16, device=dev) for _ in packed]
+    _check(load().kvq_dequantize_batch(_ptrs(packed, "packed"), _ptrs(scales, "scales"), _ptrs(amax, "amax"), n,
+                                       numel, int(head_dim), _ptrs(ys, "y"), _stream(stream, dev)))
+    return ys
+
+
+def kvq_quantize_dequantize(x: torch.Tensor, head_dim: int | None = None, rule="static_6",
+                            amax_in: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
+                            packed: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                            y: torch.Tensor | None = None, codes: bool = True, stream=None):
+    """Fused round trip: returns (y, packed, scales, amax); with codes=False only y (and
+    amax) are written and packed/scales are None."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    n = x.numel()
+    head_dim = int(head_dim or x.shape[-1])
+    dev = x.device
+    if codes:
+        packed = packed if packed is not None else torch.empty(n // 2, dtype=torch.uint8, device=dev)
+        scales = scales if scales is not None else torch.empty(n // BLOCK, dtype=torch.uint8, device=dev)
+    else:
+        packed = scales = None
+    if y is None:
+        y = torch.empty_like(x)
+    if amax_out is None and amax_in is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(load().kvq_quantize_dequantize(_dev(x, "x"), n, head_dim, _rule(rule),
+                                          None if amax_in is None else _dev(amax_in, "amax_in"),
+                                          None if amax_out is None else _dev(amax_out, "amax_out"),
+                                          None if packed is None else _dev(packed, "packed"),
+                                          None if scales is None else _dev(scales, "scales"), _dev(y, "y"),
+                                          _stream(stream, dev)))
+    return y, packed, scales, (amax_out if amax_out is not None else amax_in)
 
 
 class KVCache:

@@ -7,18 +7,19 @@
 // Parameters Reference") is restated in include/kvq.h. This file holds the kernels and
 // the C ABI around them.
 //
-// Kernels (all bandwidth-bound streaming passes; no tensor cores, no shared-memory
-// staging: every access is a fully coalesced 256-bit or narrower vector access):
+// Kernels (streaming passes; no tensor cores, no shared-memory staging of data: every
+// access is a fully coalesced 256-bit or narrower vector access):
 //   zero_kernel      clears the amax slots a quantize is about to reduce into.
 //   amax_kernel      max |x| over each tensor: 256-bit loads, per-lane u16x2 max on the
 //                    bf16 bit patterns, warp redux, one atomic max per CTA.
 //   quantize_kernel  one thread per BPT blocks: one 256-bit load per block, block amax,
 //                    e4m3 scale(s) by the rule, e2m1 codes via cvt.satfinite.e2m1x2,
-//                    8 bytes of codes + 1 scale byte per block stored.
+//                    8 bytes of codes + 1 scale byte per block stored; in its round-trip
+//                    modes it also writes the bf16 reconstruction (fake quantization).
 //   dequant_kernel   the mirror image: 8 bytes + 1 scale byte -> one 256-bit bf16 store
 //                    per block; the cache form looks up each block's chunk amax.
-// Every kernel takes a batch of tensors (blockIdx.y = tensor), so one launch covers
-// every layer's K and V of an append or a read.
+// Every kernel takes a batch of tensors, so one launch covers every layer's K and V of
+// an append or a read.
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -51,11 +52,16 @@ struct ZeroBatch {
 
 struct QuantTensor {
     const void* x;
-    uint8_t* packed;
-    uint8_t* scales;
+    uint8_t* packed;    // codes out (unused in MODE kYOnly)
+    uint8_t* scales;    // scale codes out (unused in MODE kYOnly)
     const float* amax;  // amax used for this tensor
     float* amax_copy;   // when non-null, also receives *amax
+    void* y;            // bf16 reconstruction out (MODE kCodesAndY, kYOnly)
 };
+
+// What quantize_kernel writes: the codes, the codes and the bf16 round trip, or the
+// round trip alone ("fake quantization").
+enum QuantMode { kCodes = 0, kCodesAndY = 1, kYOnly = 2 };
 
 struct QuantBatch {
     QuantTensor t[kMaxBatch];
@@ -274,12 +280,35 @@ __device__ __forceinline__ uint32_t quantize_block(const uint32_t (&w)[8], const
     }
 }
 
+// One block: 8 code bytes (two words) and its decoded scale S -> 16 bf16 (eight words),
+// y = bf16_rne(value * S).
+__device__ __forceinline__ void bf16_from_codes(uint32_t q0, uint32_t q1, float S, uint32_t (&y)[8])
+{
+    const uint64_t S2 = f32x2_pack(S, S);
+    float v[8];
+    e2m1x8_to_f32(q0, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float lo, hi;
+        f32x2_unpack(f32x2_mul(f32x2_pack(v[2 * j], v[2 * j + 1]), S2), lo, hi);
+        y[j] = bf16x2_from_f32(hi, lo);
+    }
+    e2m1x8_to_f32(q1, v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        float lo, hi;
+        f32x2_unpack(f32x2_mul(f32x2_pack(v[2 * j], v[2 * j + 1]), S2), lo, hi);
+        y[4 + j] = bf16x2_from_f32(hi, lo);
+    }
+}
+
 // Unit u of a tensor: blocks [u*BPT, u*BPT + BPT) clipped to n_blocks.
-template <int RULE, int BPT, bool MARK>
+template <int RULE, int BPT, bool MARK, int MODE>
 __device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, uint64_t n_blocks,
                                               const Quotients& qt, const ScaleTables& tab)
 {
     const char* x = static_cast<const char*>(T.x);
+    char* y = static_cast<char*>(T.y);
     const uint64_t b0 = u * BPT;
     if (BPT == 2 && b0 + 1 < n_blocks) {
         uint32_t w0[8], w1[8];
@@ -288,23 +317,41 @@ __device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, 
         uint32_t q0, q1, q2, q3;
         const uint32_t c0 = quantize_block<RULE, MARK>(w0, qt, tab, q0, q1);
         const uint32_t c1 = quantize_block<RULE, MARK>(w1, qt, tab, q2, q3);
-        st_v4(T.packed + b0 * 8, q0, q1, q2, q3);
-        *reinterpret_cast<uint16_t*>(T.scales + b0) = static_cast<uint16_t>(c0 | (c1 << 8));
+        if (MODE != kYOnly) {
+            st_v4(T.packed + b0 * 8, q0, q1, q2, q3);
+            *reinterpret_cast<uint16_t*>(T.scales + b0) = static_cast<uint16_t>(c0 | (c1 << 8));
+        }
+        if (MODE != kCodes) {
+            uint32_t yy[8];
+            bf16_from_codes(q0, q1, tab.S[c0], yy);
+            st_v8(y + b0 * 32, yy);
+            bf16_from_codes(q2, q3, tab.S[c1], yy);
+            st_v8(y + b0 * 32 + 32, yy);
+        }
     } else {  // BPT == 1, or the odd last block of a pair unit
         uint32_t w0[8];
         ld_nc_v8(x + b0 * 32, w0);
         uint32_t q0, q1;
         const uint32_t c0 = quantize_block<RULE, MARK>(w0, qt, tab, q0, q1);
-        st_v2(T.packed + b0 * 8, q0, q1);
-        T.scales[b0] = static_cast<uint8_t>(c0);
+        if (MODE != kYOnly) {
+            st_v2(T.packed + b0 * 8, q0, q1);
+            T.scales[b0] = static_cast<uint8_t>(c0);
+        }
+        if (MODE != kCodes) {
+            uint32_t yy[8];
+            bf16_from_codes(q0, q1, tab.S[c0], yy);
+            st_v8(y + b0 * 32, yy);
+        }
     }
 }
 
 // grid (tiles, tensors), one unit of BPT blocks per thread. The tiles and tensors are
 // walked in the reverse of amax_kernel's order, so the data amax_kernel read last (still
 // in L2) is quantized first. With BPT = 2 the packed pointer must be 16-byte and the
-// scale pointer 2-byte aligned.
-template <int RULE, int BPT>
+// scale pointer 2-byte aligned. MODE selects the outputs (QuantMode); the round trip
+// y = bf16_rne(value * S) is the same arithmetic as dequant_kernel, so it is bit-equal
+// to quantizing and then dequantizing.
+template <int RULE, int BPT, int MODE>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
 {
     __shared__ ScaleTables tab;
@@ -322,33 +369,17 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
     if (u * BPT >= B.n_blocks)
         return;
     if (qt.markstein)
-        quantize_unit<RULE, BPT, true>(T, u, B.n_blocks, qt, tab);
+        quantize_unit<RULE, BPT, true, MODE>(T, u, B.n_blocks, qt, tab);
     else
-        quantize_unit<RULE, BPT, false>(T, u, B.n_blocks, qt, tab);
+        quantize_unit<RULE, BPT, false, MODE>(T, u, B.n_blocks, qt, tab);
 }
 
-// One block: 8 code bytes (two words) and its scale -> 16 bf16 (eight words).
+// One block: 8 code bytes and its scale code under global scale gs -> 16 bf16.
 __device__ __forceinline__ void dequant_block(uint32_t q0, uint32_t q1, uint32_t c, float gs, uint32_t (&y)[8])
 {
     float S, unused;
     e4m3x2_to_f32(c & 0xFFu, S, unused);
-    S = __fmul_rn(S, gs);
-    const uint64_t S2 = f32x2_pack(S, S);
-    float v[8];
-    e2m1x8_to_f32(q0, v);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float lo, hi;
-        f32x2_unpack(f32x2_mul(f32x2_pack(v[2 * j], v[2 * j + 1]), S2), lo, hi);
-        y[j] = bf16x2_from_f32(hi, lo);
-    }
-    e2m1x8_to_f32(q1, v);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float lo, hi;
-        f32x2_unpack(f32x2_mul(f32x2_pack(v[2 * j], v[2 * j + 1]), S2), lo, hi);
-        y[4 + j] = bf16x2_from_f32(hi, lo);
-    }
+    bf16_from_codes(q0, q1, __fmul_rn(S, gs), y);
 }
 
 // grid (tiles, chunks, tensors). Each CTA lies inside one chunk, so its amax (and global
@@ -450,7 +481,38 @@ kvq_status check_shape(int64_t n_elems, int32_t head_dim)
 
 // Quantize a batch of equally sized tensors whose amax slots are given. When
 // compute_amax, the slots are cleared and reduced first.
-kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s)
+template <int RULE, int BPT>
+void launch_quantize_mode(int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+{
+    if (mode == kCodes)
+        quantize_kernel<RULE, BPT, kCodes><<<grid, kThreads, 0, s>>>(qb);
+    else if (mode == kCodesAndY)
+        quantize_kernel<RULE, BPT, kCodesAndY><<<grid, kThreads, 0, s>>>(qb);
+    else
+        quantize_kernel<RULE, BPT, kYOnly><<<grid, kThreads, 0, s>>>(qb);
+}
+
+template <int RULE>
+void launch_quantize_bpt(int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+{
+    if (bpt == 2)
+        launch_quantize_mode<RULE, 2>(mode, grid, qb, s);
+    else
+        launch_quantize_mode<RULE, 1>(mode, grid, qb, s);
+}
+
+void launch_quantize(kvq_scale_rule rule, int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+{
+    if (rule == KVQ_RULE_STATIC_6)
+        launch_quantize_bpt<KVQ_RULE_STATIC_6>(bpt, mode, grid, qb, s);
+    else if (rule == KVQ_RULE_STATIC_4)
+        launch_quantize_bpt<KVQ_RULE_STATIC_4>(bpt, mode, grid, qb, s);
+    else
+        launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, grid, qb, s);
+}
+
+kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s,
+                        int mode = kCodes)
 {
     if (n == 0 || qb.n_blocks == 0)
         return KVQ_OK;
@@ -473,24 +535,11 @@ kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scal
             return st;
     }
     bool pairs = true;
-    for (int i = 0; i < n; ++i)
-        pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
+    if (mode != kYOnly)
+        for (int i = 0; i < n; ++i)
+            pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
     const dim3 grid(tiles(pairs ? (qb.n_blocks + 1) / 2 : qb.n_blocks), n);
-    if (pairs) {
-        if (rule == KVQ_RULE_STATIC_6)
-            quantize_kernel<KVQ_RULE_STATIC_6, 2><<<grid, kThreads, 0, s>>>(qb);
-        else if (rule == KVQ_RULE_STATIC_4)
-            quantize_kernel<KVQ_RULE_STATIC_4, 2><<<grid, kThreads, 0, s>>>(qb);
-        else
-            quantize_kernel<KVQ_RULE_MSE, 2><<<grid, kThreads, 0, s>>>(qb);
-    } else {
-        if (rule == KVQ_RULE_STATIC_6)
-            quantize_kernel<KVQ_RULE_STATIC_6, 1><<<grid, kThreads, 0, s>>>(qb);
-        else if (rule == KVQ_RULE_STATIC_4)
-            quantize_kernel<KVQ_RULE_STATIC_4, 1><<<grid, kThreads, 0, s>>>(qb);
-        else
-            quantize_kernel<KVQ_RULE_MSE, 1><<<grid, kThreads, 0, s>>>(qb);
-    }
+    launch_quantize(rule, pairs ? 2 : 1, mode, grid, qb, s);
     return check_launch("quantize_kernel");
 }
 
@@ -550,65 +599,163 @@ using namespace kvq;
 
 extern "C" {
 
-kvq_status kvq_quantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
-                        const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
-                        kvq_stream_t stream)
+}  // extern "C"
+
+namespace kvq {
+
+// Shared body of kvq_quantize, kvq_quantize_batch and kvq_quantize_dequantize: n
+// equally sized tensors. amax_in null: each tensor's amax is computed into amax_out[i].
+// amax_in given: amax_in[i] is used and copied to amax_out[i] when that is given too.
+kvq_status quantize_impl(const char* what, const void* const* xs, int32_t n, int64_t n_elems, int32_t head_dim,
+                         kvq_scale_rule rule, const float* const* amax_in, float* const* amax_out,
+                         uint8_t* const* packed, uint8_t* const* scales, void* const* ys, int mode,
+                         cudaStream_t s)
 {
     kvq_status st;
     if ((st = check_shape(n_elems, head_dim)) != KVQ_OK || (st = check_rule(rule)) != KVQ_OK)
         return st;
+    if (n < 0)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: negative tensor count", what);
+    if (n == 0)
+        return ok();
     if (amax_in == nullptr && amax_out == nullptr)
-        return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize: amax_in and amax_out are both null");
-    if (n_elems > 0 && (x == nullptr || packed == nullptr || scales == nullptr))
-        return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize: null tensor pointer");
-    if (!aligned(x, 32) || !aligned(packed, 8) || !aligned(amax_in, 4) || !aligned(amax_out, 4))
-        return fail(KVQ_ERR_MISALIGNED, "kvq_quantize: x must be 32-byte, packed 8-byte, amax 4-byte aligned");
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        return fail(KVQ_ERR_INVALID_ARG, "%s: amax_in and amax_out are both null", what);
+    if (xs == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: null xs array", what);
+    if (mode != kYOnly && (packed == nullptr || scales == nullptr))
+        return fail(KVQ_ERR_INVALID_ARG, "%s: null packed / scales array", what);
+    if (mode != kCodes && ys == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "%s: null y array", what);
+    for (int i = 0; i < n; ++i) {
+        const float* ain = amax_in ? amax_in[i] : nullptr;
+        float* aout = amax_out ? amax_out[i] : nullptr;
+        if (ain == nullptr && aout == nullptr)
+            return fail(KVQ_ERR_INVALID_ARG, "%s: amax_in and amax_out are both null", what);
+        if (amax_in != nullptr && ain == nullptr)
+            return fail(KVQ_ERR_INVALID_ARG, "%s: amax_in given for some tensors only", what);
+        if (n_elems > 0 && (xs[i] == nullptr || (mode != kYOnly && (packed[i] == nullptr || scales[i] == nullptr)) ||
+                            (mode != kCodes && ys[i] == nullptr)))
+            return fail(KVQ_ERR_INVALID_ARG, "%s: null tensor pointer", what);
+        if (!aligned(xs[i], 32) || (mode != kYOnly && !aligned(packed[i], 8)) || (mode != kCodes && !aligned(ys[i], 32)) ||
+            !aligned(ain, 4) || !aligned(aout, 4))
+            return fail(KVQ_ERR_MISALIGNED, "%s: x and y must be 32-byte, packed 8-byte, amax 4-byte aligned", what);
+    }
     if (n_elems == 0) {
-        // amax of an empty tensor is 0; a given amax is passed through
-        if (amax_out != nullptr) {
-            cudaError_t e = amax_in ? cudaMemcpyAsync(amax_out, amax_in, 4, cudaMemcpyDeviceToDevice, s)
-                                    : cudaMemsetAsync(amax_out, 0, 4, s);
+        // the amax of an empty tensor is 0; a given amax is passed through
+        for (int i = 0; i < n; ++i) {
+            float* aout = amax_out ? amax_out[i] : nullptr;
+            const float* ain = amax_in ? amax_in[i] : nullptr;
+            if (aout == nullptr)
+                continue;
+            cudaError_t e = ain ? cudaMemcpyAsync(aout, ain, 4, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(aout, 0, 4, s);
             if (e != cudaSuccess)
-                return fail(KVQ_ERR_CUDA, "kvq_quantize: %s", cudaGetErrorString(e));
+                return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
         }
         return ok();
     }
-    QuantBatch qb{};
-    qb.n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
-    qb.t[0].x = x;
-    qb.t[0].packed = packed;
-    qb.t[0].scales = scales;
-    qb.t[0].amax = amax_in ? amax_in : amax_out;
-    qb.t[0].amax_copy = (amax_in && amax_out && amax_out != amax_in) ? amax_out : nullptr;
-    if ((st = run_quantize(qb, 1, amax_in == nullptr, rule, s)) != KVQ_OK)
-        return st;
+    const uint64_t n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
+    for (int base = 0; base < n; base += kMaxBatch) {
+        const int m = n - base < kMaxBatch ? n - base : kMaxBatch;
+        QuantBatch qb{};
+        qb.n_blocks = n_blocks;
+        for (int i = 0; i < m; ++i) {
+            const int j = base + i;
+            const float* ain = amax_in ? amax_in[j] : nullptr;
+            float* aout = amax_out ? amax_out[j] : nullptr;
+            qb.t[i].x = xs[j];
+            qb.t[i].packed = mode != kYOnly ? packed[j] : nullptr;
+            qb.t[i].scales = mode != kYOnly ? scales[j] : nullptr;
+            qb.t[i].amax = ain ? ain : aout;
+            qb.t[i].amax_copy = (ain && aout && aout != ain) ? aout : nullptr;
+            qb.t[i].y = mode != kCodes ? ys[j] : nullptr;
+        }
+        if ((st = run_quantize(qb, m, amax_in == nullptr, rule, s, mode)) != KVQ_OK)
+            return st;
+    }
     return ok();
+}
+
+kvq_status dequantize_impl(const uint8_t* const* packed, const uint8_t* const* scales, const float* const* amax,
+                           int32_t n, int64_t n_elems, int32_t head_dim, void* const* ys, cudaStream_t s)
+{
+    kvq_status st;
+    if ((st = check_shape(n_elems, head_dim)) != KVQ_OK)
+        return st;
+    if (n < 0)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize: negative tensor count");
+    if (n == 0 || n_elems == 0)
+        return ok();
+    if (packed == nullptr || scales == nullptr || amax == nullptr || ys == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize: null host array");
+    for (int i = 0; i < n; ++i) {
+        if (packed[i] == nullptr || scales[i] == nullptr || amax[i] == nullptr || ys[i] == nullptr)
+            return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize: null pointer");
+        if (!aligned(ys[i], 32) || !aligned(packed[i], 8) || !aligned(amax[i], 4))
+            return fail(KVQ_ERR_MISALIGNED, "kvq_dequantize: y must be 32-byte, packed 8-byte, amax 4-byte aligned");
+    }
+    for (int base = 0; base < n; base += kMaxBatch) {
+        const int m = n - base < kMaxBatch ? n - base : kMaxBatch;
+        DequantBatch db{};
+        db.blk_lo = 0;
+        db.blk_hi = static_cast<uint64_t>(n_elems) / kBlock;
+        db.blocks_per_chunk = db.blk_hi;  // one chunk: the tensor
+        for (int i = 0; i < m; ++i) {
+            db.t[i].packed = packed[base + i];
+            db.t[i].scales = scales[base + i];
+            db.t[i].amax = amax[base + i];
+            db.t[i].y = ys[base + i];
+        }
+        if ((st = run_dequantize(db, m, s)) != KVQ_OK)
+            return st;
+    }
+    return ok();
+}
+
+}  // namespace kvq
+
+extern "C" {
+
+kvq_status kvq_quantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
+                        const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
+                        kvq_stream_t stream)
+{
+    return quantize_impl("kvq_quantize", &x, 1, n_elems, head_dim, rule, amax_in ? &amax_in : nullptr,
+                         amax_out ? &amax_out : nullptr, &packed, &scales, nullptr, kCodes,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_quantize_batch(const void* const* xs, int32_t n_tensors, int64_t n_elems, int32_t head_dim,
+                              kvq_scale_rule rule, const float* const* amax_in, float* const* amax_out,
+                              uint8_t* const* packed, uint8_t* const* scales, kvq_stream_t stream)
+{
+    return quantize_impl("kvq_quantize_batch", xs, n_tensors, n_elems, head_dim, rule, amax_in, amax_out, packed,
+                         scales, nullptr, kCodes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_quantize_dequantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
+                                   const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
+                                   void* y, kvq_stream_t stream)
+{
+    if ((packed == nullptr) != (scales == nullptr))
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize_dequantize: packed and scales must be both given or both null");
+    const int mode = packed ? kCodesAndY : kYOnly;
+    return quantize_impl("kvq_quantize_dequantize", &x, 1, n_elems, head_dim, rule, amax_in ? &amax_in : nullptr,
+                         amax_out ? &amax_out : nullptr, &packed, &scales, &y, mode,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+kvq_status kvq_dequantize_batch(const uint8_t* const* packed, const uint8_t* const* scales, const float* const* amax,
+                                int32_t n_tensors, int64_t n_elems, int32_t head_dim, void* const* ys,
+                                kvq_stream_t stream)
+{
+    return dequantize_impl(packed, scales, amax, n_tensors, n_elems, head_dim, ys,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const float* amax, int64_t n_elems,
                           int32_t head_dim, void* y, kvq_stream_t stream)
 {
-    kvq_status st;
-    if ((st = check_shape(n_elems, head_dim)) != KVQ_OK)
-        return st;
-    if (n_elems == 0)
-        return ok();
-    if (packed == nullptr || scales == nullptr || amax == nullptr || y == nullptr)
-        return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize: null pointer");
-    if (!aligned(y, 32) || !aligned(packed, 8) || !aligned(amax, 4))
-        return fail(KVQ_ERR_MISALIGNED, "kvq_dequantize: y must be 32-byte, packed 8-byte, amax 4-byte aligned");
-    DequantBatch db{};
-    db.blk_lo = 0;
-    db.blk_hi = static_cast<uint64_t>(n_elems) / kBlock;
-    db.blocks_per_chunk = db.blk_hi;  // one chunk: the tensor
-    db.t[0].packed = packed;
-    db.t[0].scales = scales;
-    db.t[0].amax = amax;
-    db.t[0].y = y;
-    if ((st = run_dequantize(db, 1, reinterpret_cast<cudaStream_t>(stream))) != KVQ_OK)
-        return st;
-    return ok();
+    return dequantize_impl(&packed, &scales, &amax, 1, n_elems, head_dim, &y, reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_append_batch(const kvq_cache* caches, const int64_t* row_offsets, const void* const* xs,

@@ -22,7 +22,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("kvq_quantize", "kvq_dequantize", "kvq_append", "kvq_append_batch", "kvq_dequantize_cache",
+    for must in ("kvq_quantize", "kvq_dequantize", "kvq_quantize_batch", "kvq_dequantize_batch",
+                 "kvq_quantize_dequantize", "kvq_append", "kvq_append_batch", "kvq_dequantize_cache",
                  "kvq_dequantize_cache_batch", "kvq_cache_bytes", "kvq_status_string", "kvq_last_error"):
         assert must in names
 
@@ -78,6 +79,15 @@ def test_invalid_arguments_rejected_before_any_launch():
     assert lib.kvq_dequantize(_fake(A), _fake(A), _fake(A), 128, 128, _fake(A + 2), None) == 2
     # too large
     assert lib.kvq_quantize(_fake(A), (1 << 37), 128, 0, None, _fake(A), _fake(A), _fake(A), None) == 3
+    # round trip: packed and scales must come together; y alignment
+    assert lib.kvq_quantize_dequantize(_fake(A), 128, 128, 0, None, _fake(A), _fake(A), None, _fake(A), None) == 1
+    assert lib.kvq_quantize_dequantize(_fake(A), 128, 128, 0, None, _fake(A), None, None, _fake(A + 16), None) == 2
+    # batch: amax_in given for some tensors only
+    xs = (ctypes.c_void_p * 2)(A, A)
+    ain = (ctypes.c_void_p * 2)(A, None)
+    outs = (ctypes.c_void_p * 2)(A, A)
+    assert lib.kvq_quantize_batch(xs, 2, 128, 128, 0, ain, None, outs, outs, None) == 1
+    assert lib.kvq_quantize_batch(xs, -1, 128, 128, 0, None, outs, outs, outs, None) == 1
 
 
 def _cache(capacity_rows=64, rows_per_chunk=16, head_dim=128, base=1 << 40):

@@ -276,3 +276,63 @@ def test_cache_capacity_error_leaves_cache_untouched():
     assert e.value.status == 4
     torch.cuda.synchronize()
     assert not c.packed.any() and not c.scales.any()
+
+
+# ---------------------------------------------------------------- batched and fused entry points
+
+@pytest.mark.parametrize("rule", RULES)
+def test_quantize_batch_matches_oracle_per_tensor(orc, rule):
+    """K and V (and a third tensor) in one set of launches, each with its own amax."""
+    xs = [inputs.layer_kv(kv, heads=3, tokens=331, device="cuda") for kv in (0, 1)]
+    xs.append(inputs.normal(tuple(xs[0].shape), seed=77, device="cuda") * 1e-3)
+    p, s, a = kvq.kvq_quantize_batch(xs, 128, rule)
+    ys = kvq.kvq_dequantize_batch(p, s, a, 128)
+    torch.cuda.synchronize()
+    for i, x in enumerate(xs):
+        pe, se, ae = orc.quantize(bits(x), 128, rule)
+        assert float(a[i][0]) == ae
+        assert_same(s[i].cpu().numpy(), se, f"scales t{i}")
+        assert_same(p[i].cpu().numpy(), pe, f"packed t{i}")
+        assert_same(bits(ys[i]), orc.dequantize(pe, se, ae, 128), f"dequant t{i}")
+
+
+def test_batches_above_the_launch_limit_are_split(orc):
+    n = kvq.MAX_BATCH + 7
+    xs = [inputs.normal((3, 128), seed=500 + i, device="cuda") * (i + 1) for i in range(n)]
+    p, s, a = kvq.kvq_quantize_batch(xs, 128, "mse")
+    ys = kvq.kvq_dequantize_batch(p, s, a, 128)
+    torch.cuda.synchronize()
+    for i in (0, kvq.MAX_BATCH - 1, kvq.MAX_BATCH, n - 1):
+        pe, se, ae = orc.quantize(bits(xs[i]), 128, "mse")
+        assert float(a[i][0]) == ae
+        assert_same(p[i].cpu().numpy(), pe, f"packed t{i}")
+        assert_same(bits(ys[i]), orc.dequantize(pe, se, ae, 128), f"dequant t{i}")
+
+
+@pytest.mark.parametrize("codes", [True, False])
+@pytest.mark.parametrize("rule", RULES)
+def test_fused_round_trip_equals_quantize_then_dequantize(orc, rule, codes):
+    cases = [inputs.single_k("cuda"), inputs.normal((7, 48), seed=3, device="cuda"),
+             inputs.layer_kv(1, heads=2, tokens=257, device="cuda")]
+    for x in cases:
+        D = x.shape[-1]
+        y, p, s, a = kvq.kvq_quantize_dequantize(x, D, rule, codes=codes)
+        torch.cuda.synchronize()
+        pe, se, ae = orc.quantize(bits(x), D, rule)
+        assert float(a[0]) == ae
+        assert_same(bits(y), orc.dequantize(pe, se, ae, D), f"round trip {tuple(x.shape)}")
+        if codes:
+            assert_same(p.cpu().numpy(), pe, "packed")
+            assert_same(s.cpu().numpy(), se, "scales")
+        else:
+            assert p is None and s is None
+
+
+def test_fused_round_trip_with_amax_in(orc):
+    x = inputs.normal((129, 128), seed=12, device="cuda")
+    for given in (float(x.abs().max().float()) / 4, 0.0):
+        amax_in = torch.tensor([given], device="cuda")
+        y, _, _, _ = kvq.kvq_quantize_dequantize(x, 128, "mse", amax_in=amax_in, codes=False)
+        torch.cuda.synchronize()
+        pe, se, _ = orc.quantize(bits(x), 128, "mse", amax_in=given)
+        assert_same(bits(y), orc.dequantize(pe, se, given, 128), f"round trip amax_in={given}")

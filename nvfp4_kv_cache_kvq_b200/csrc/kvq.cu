@@ -92,6 +92,7 @@ constexpr int kAmaxIters = 4;  // blocks per thread in amax_kernel
 
 __global__ void __launch_bounds__(64) zero_kernel(const ZeroBatch z)
 {
+    pdl_begin();
     int i = threadIdx.x;
     if (i < z.n)
         *z.out[i] = 0u;
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(64) zero_kernel(const ZeroBatch z)
 // grid (tiles, tensors); a tile is kThreads * kAmaxIters blocks.
 __global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxBatch B)
 {
+    pdl_begin();
     const char* x = static_cast<const char*>(B.x[blockIdx.y]);
     const uint64_t base = static_cast<uint64_t>(blockIdx.x) * (kThreads * kAmaxIters) + threadIdx.x;
     uint32_t w[kAmaxIters][8];
@@ -354,6 +356,7 @@ __device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, 
 template <int RULE, int BPT, int MODE>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
 {
+    pdl_begin();
     __shared__ ScaleTables tab;
     const QuantTensor& T = B.t[gridDim.y - 1 - blockIdx.y];
     const float amax = __ldg(T.amax);
@@ -388,6 +391,7 @@ __device__ __forceinline__ void dequant_block(uint32_t q0, uint32_t q1, uint32_t
 template <int BPT>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(const DequantBatch B)
 {
+    pdl_begin();
     const DequantTensor& T = B.t[blockIdx.z];
     const uint64_t chunk = B.chunk0 + blockIdx.y;
     const uint64_t c_lo = chunk * B.blocks_per_chunk;
@@ -443,11 +447,30 @@ kvq_status ok()
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-kvq_status check_launch(const char* what)
+// Launch with programmatic stream serialization (see pdl_begin): the kernel may be
+// scheduled while the previous grid on the stream drains, and waits for it on entry.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, unsigned threads, cudaStream_t s, Args... args)
 {
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+kvq_status launched(cudaError_t e, const char* what)
+{
+    if (e != cudaSuccess) {
+        cudaGetLastError();
         return fail(KVQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    }
     return KVQ_OK;
 }
 
@@ -482,33 +505,31 @@ kvq_status check_shape(int64_t n_elems, int32_t head_dim)
 // Quantize a batch of equally sized tensors whose amax slots are given. When
 // compute_amax, the slots are cleared and reduced first.
 template <int RULE, int BPT>
-void launch_quantize_mode(int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+cudaError_t launch_quantize_mode(int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
 {
+    cudaError_t e;
     if (mode == kCodes)
-        quantize_kernel<RULE, BPT, kCodes><<<grid, kThreads, 0, s>>>(qb);
+        e = launch(quantize_kernel<RULE, BPT, kCodes>, grid, kThreads, s, qb);
     else if (mode == kCodesAndY)
-        quantize_kernel<RULE, BPT, kCodesAndY><<<grid, kThreads, 0, s>>>(qb);
+        e = launch(quantize_kernel<RULE, BPT, kCodesAndY>, grid, kThreads, s, qb);
     else
-        quantize_kernel<RULE, BPT, kYOnly><<<grid, kThreads, 0, s>>>(qb);
+        e = launch(quantize_kernel<RULE, BPT, kYOnly>, grid, kThreads, s, qb);
+    return e;
 }
 
 template <int RULE>
-void launch_quantize_bpt(int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+cudaError_t launch_quantize_bpt(int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
 {
-    if (bpt == 2)
-        launch_quantize_mode<RULE, 2>(mode, grid, qb, s);
-    else
-        launch_quantize_mode<RULE, 1>(mode, grid, qb, s);
+    return bpt == 2 ? launch_quantize_mode<RULE, 2>(mode, grid, qb, s) : launch_quantize_mode<RULE, 1>(mode, grid, qb, s);
 }
 
-void launch_quantize(kvq_scale_rule rule, int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+cudaError_t launch_quantize(kvq_scale_rule rule, int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
 {
     if (rule == KVQ_RULE_STATIC_6)
-        launch_quantize_bpt<KVQ_RULE_STATIC_6>(bpt, mode, grid, qb, s);
-    else if (rule == KVQ_RULE_STATIC_4)
-        launch_quantize_bpt<KVQ_RULE_STATIC_4>(bpt, mode, grid, qb, s);
-    else
-        launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, grid, qb, s);
+        return launch_quantize_bpt<KVQ_RULE_STATIC_6>(bpt, mode, grid, qb, s);
+    if (rule == KVQ_RULE_STATIC_4)
+        return launch_quantize_bpt<KVQ_RULE_STATIC_4>(bpt, mode, grid, qb, s);
+    return launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, grid, qb, s);
 }
 
 kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s,
@@ -527,11 +548,10 @@ kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scal
         }
         z.n = n;
         ab.n_blocks = qb.n_blocks;
-        zero_kernel<<<1, 64, 0, s>>>(z);
-        if ((st = check_launch("zero_kernel")) != KVQ_OK)
+        if ((st = launched(launch(zero_kernel, dim3(1), 64, s, z), "zero_kernel")) != KVQ_OK)
             return st;
-        amax_kernel<<<dim3(tiles(qb.n_blocks, kAmaxIters), n), kThreads, 0, s>>>(ab);
-        if ((st = check_launch("amax_kernel")) != KVQ_OK)
+        if ((st = launched(launch(amax_kernel, dim3(tiles(qb.n_blocks, kAmaxIters), n), kThreads, s, ab),
+                           "amax_kernel")) != KVQ_OK)
             return st;
     }
     bool pairs = true;
@@ -539,8 +559,7 @@ kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scal
         for (int i = 0; i < n; ++i)
             pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
     const dim3 grid(tiles(pairs ? (qb.n_blocks + 1) / 2 : qb.n_blocks), n);
-    launch_quantize(rule, pairs ? 2 : 1, mode, grid, qb, s);
-    return check_launch("quantize_kernel");
+    return launched(launch_quantize(rule, pairs ? 2 : 1, mode, grid, qb, s), "quantize_kernel");
 }
 
 // Dequantize blocks [blk_lo, blk_hi) of n equally laid-out tensors; packed/scales point at
@@ -561,11 +580,9 @@ kvq_status run_dequantize(DequantBatch db, int n, cudaStream_t s)
         const uint64_t nc = (last - c0 + 1) < 65535 ? (last - c0 + 1) : 65535;
         db.chunk0 = c0;
         const dim3 grid(gx, static_cast<unsigned>(nc), n);
-        if (pairs)
-            dequant_kernel<2><<<grid, kThreads, 0, s>>>(db);
-        else
-            dequant_kernel<1><<<grid, kThreads, 0, s>>>(db);
-        kvq_status st = check_launch("dequant_kernel");
+        kvq_status st = launched(pairs ? launch(dequant_kernel<2>, grid, kThreads, s, db)
+                                       : launch(dequant_kernel<1>, grid, kThreads, s, db),
+                                 "dequant_kernel");
         if (st != KVQ_OK)
             return st;
     }

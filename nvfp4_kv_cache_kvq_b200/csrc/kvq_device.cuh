@@ -11,6 +11,17 @@
 
 namespace kvq {
 
+// Programmatic dependent launch (sm_90+). Every kernel of the library starts with
+// pdl_begin(): it waits until the grid launched before it on the stream has completed and
+// its writes are visible (a no-op when the launch carried no programmatic dependency),
+// then lets the next grid be scheduled. The next grid's launch latency thus overlaps this
+// grid's tail, while its own pdl_begin() still orders every memory access after ours.
+__device__ __forceinline__ void pdl_begin()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 32 bytes (one 16-element bf16 block) from read-only global memory, not kept in L1.
 __device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&w)[8])
 {

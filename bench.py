@@ -254,20 +254,20 @@ class Layer:
         self.kvq = kvq
 
     def segments(self):
-        kvq = self.kvq
+        kvq, m = self.kvq, len(self.x)
 
         def q():
-            for i in range(2):
-                kvq.kvq_quantize(self.x[i], self.D, self.rule, amax_out=self.a[i], packed=self.p[i], scales=self.s[i])
+            kvq.kvq_quantize_batch(self.x, self.D, self.rule, amax_out=self.a[:m], packed=self.p[:m],
+                                   scales=self.s[:m])
 
         def d():
-            for i in range(2):
-                kvq.kvq_dequantize(self.p[i], self.s[i], self.a[i], self.D, y=self.y[i])
-        return [Segment("quantize", q, 6, 2 * self.n * (B_AMAX + B_QUANT), h2d=tuple(self.x)),
-                Segment("dequant", d, 2, 2 * self.n * B_DEQUANT)]
+            kvq.kvq_dequantize_batch(self.p[:m], self.s[:m], self.a[:m], self.D, ys=self.y[:m])
+        return [Segment("quantize", q, 3, m * self.n * (B_AMAX + B_QUANT), h2d=tuple(self.x)),
+                Segment("dequant", d, 1, m * self.n * B_DEQUANT)]
 
     def d2h(self):
-        return self.p + self.s + self.a + self.y
+        m = len(self.x)
+        return self.p[:m] + self.s[:m] + self.a[:m] + self.y[:m]
 
     def tokens_per_step(self):
         return self.tokens
@@ -318,14 +318,16 @@ class Cache:
         kvq, T = self.kvq, 2 * self.layers
 
         def q():
-            for t in range(T):
-                kvq.kvq_quantize(self.x[t], self.D, self.rule, amax_out=self.a[t], packed=self.p[t], scales=self.s[t])
+            kvq.kvq_quantize_batch(list(self.x), self.D, self.rule, amax_out=list(self.a), packed=list(self.p),
+                                   scales=list(self.s))
 
         def d():
-            for t in range(T):
-                kvq.kvq_dequantize(self.p[t], self.s[t], self.a[t], self.D, y=self.y[t % 2])
-        return [Segment("quantize", q, 3 * T, T * self.n * (B_AMAX + B_QUANT), h2d=(self.x,)),
-                Segment("dequant", d, T, T * self.n * B_DEQUANT)]
+            for l in range(self.layers):
+                kvq.kvq_dequantize_batch([self.p[2 * l], self.p[2 * l + 1]], [self.s[2 * l], self.s[2 * l + 1]],
+                                         [self.a[2 * l], self.a[2 * l + 1]], self.D, ys=[self.y[0], self.y[1]])
+        return [Segment("quantize", q, 3 * math.ceil(T / self.kvq.MAX_BATCH), T * self.n * (B_AMAX + B_QUANT),
+                        h2d=(self.x,)),
+                Segment("dequant", d, self.layers, T * self.n * B_DEQUANT)]
 
     def d2h(self):
         return [self.p, self.s, self.a]
@@ -363,7 +365,7 @@ class Single(Layer):
 
     def setup(self, kvq, inputs, dev):
         Layer.setup(self, kvq, inputs, dev)
-        self.x = [inputs.normal((self.tokens, self.D), seed=2 * self.rank + kv, device=dev) for kv in (0, 1)]
+        self.x = [inputs.normal((self.tokens, self.D), seed=self.rank, device=dev)]
 
     def oracle_sample(self, orc, inputs, budget_s):
         t0, nbytes, reps = time.perf_counter(), 0.0, 0
@@ -393,7 +395,7 @@ class Sweep(Layer):
 
     def setup(self, kvq, inputs, dev):
         Layer.setup(self, kvq, inputs, dev)
-        self.x = [inputs.sweep(self.tokens, device=dev)] * 2
+        self.x = [inputs.sweep(self.tokens, device=dev)]
 
     def oracle_sample(self, orc, inputs, budget_s):
         nbytes, reps = 0.0, 0

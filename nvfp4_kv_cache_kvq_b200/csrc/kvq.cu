@@ -347,13 +347,13 @@ __device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, 
     }
 }
 
-// grid (tiles, tensors), one unit of BPT blocks per thread. The tiles and tensors are
+// grid (tiles, tensors), UPT units of BPT blocks per thread. The tiles and tensors are
 // walked in the reverse of amax_kernel's order, so the data amax_kernel read last (still
 // in L2) is quantized first. With BPT = 2 the packed pointer must be 16-byte and the
 // scale pointer 2-byte aligned. MODE selects the outputs (QuantMode); the round trip
 // y = bf16_rne(value * S) is the same arithmetic as dequant_kernel, so it is bit-equal
 // to quantizing and then dequantizing.
-template <int RULE, int BPT, int MODE>
+template <int RULE, int BPT, int MODE, int UPT = 1>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
 {
     pdl_begin();
@@ -368,13 +368,18 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
         *T.amax_copy = amax;
     build_scale_tables(tab, qt.gs);
 
-    const uint64_t u = static_cast<uint64_t>(gridDim.x - 1 - blockIdx.x) * kThreads + threadIdx.x;
-    if (u * BPT >= B.n_blocks)
-        return;
-    if (qt.markstein)
-        quantize_unit<RULE, BPT, true, MODE>(T, u, B.n_blocks, qt, tab);
-    else
-        quantize_unit<RULE, BPT, false, MODE>(T, u, B.n_blocks, qt, tab);
+    // the CTA's tile: UPT rows of kThreads consecutive units
+    const uint64_t tile = static_cast<uint64_t>(gridDim.x - 1 - blockIdx.x) * (kThreads * UPT);
+#pragma unroll 1
+    for (int i = 0; i < UPT; ++i) {
+        const uint64_t u = tile + static_cast<uint64_t>(i) * kThreads + threadIdx.x;
+        if (u * BPT >= B.n_blocks)
+            return;
+        if (qt.markstein)
+            quantize_unit<RULE, BPT, true, MODE>(T, u, B.n_blocks, qt, tab);
+        else
+            quantize_unit<RULE, BPT, false, MODE>(T, u, B.n_blocks, qt, tab);
+    }
 }
 
 // One block: 8 code bytes and its scale code under global scale gs -> 16 bf16.
@@ -504,32 +509,46 @@ kvq_status check_shape(int64_t n_elems, int32_t head_dim)
 
 // Quantize a batch of equally sized tensors whose amax slots are given. When
 // compute_amax, the slots are cleared and reduced first.
-template <int RULE, int BPT>
-cudaError_t launch_quantize_mode(int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+// Units per thread of quantize_kernel. The mse rule is instruction-bound; 8 units per
+// thread amortize the per-CTA scale tables (+4% on B200) as long as the launch keeps
+// enough CTAs to fill the GPU many times over (else the last partial wave costs more).
+// The static rules are DRAM-bound either way and keep one unit per thread.
+constexpr uint64_t kMinCtasForUpt8 = 2048;
+
+template <int RULE, int BPT, int U>
+cudaError_t launch_quantize_upt(int mode, uint64_t units, int n, const QuantBatch& qb, cudaStream_t s)
 {
-    cudaError_t e;
+    const dim3 grid(tiles(units, U), n);
     if (mode == kCodes)
-        e = launch(quantize_kernel<RULE, BPT, kCodes>, grid, kThreads, s, qb);
-    else if (mode == kCodesAndY)
-        e = launch(quantize_kernel<RULE, BPT, kCodesAndY>, grid, kThreads, s, qb);
-    else
-        e = launch(quantize_kernel<RULE, BPT, kYOnly>, grid, kThreads, s, qb);
-    return e;
+        return launch(quantize_kernel<RULE, BPT, kCodes, U>, grid, kThreads, s, qb);
+    if (mode == kCodesAndY)
+        return launch(quantize_kernel<RULE, BPT, kCodesAndY, U>, grid, kThreads, s, qb);
+    return launch(quantize_kernel<RULE, BPT, kYOnly, U>, grid, kThreads, s, qb);
+}
+
+template <int RULE, int BPT>
+cudaError_t launch_quantize_mode(int mode, uint64_t units, int n, const QuantBatch& qb, cudaStream_t s)
+{
+    if (RULE == KVQ_RULE_MSE && static_cast<uint64_t>(tiles(units, 8)) * n >= kMinCtasForUpt8)
+        return launch_quantize_upt<RULE, BPT, 8>(mode, units, n, qb, s);
+    return launch_quantize_upt<RULE, BPT, 1>(mode, units, n, qb, s);
 }
 
 template <int RULE>
-cudaError_t launch_quantize_bpt(int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+cudaError_t launch_quantize_bpt(int bpt, int mode, uint64_t units, int n, const QuantBatch& qb, cudaStream_t s)
 {
-    return bpt == 2 ? launch_quantize_mode<RULE, 2>(mode, grid, qb, s) : launch_quantize_mode<RULE, 1>(mode, grid, qb, s);
+    return bpt == 2 ? launch_quantize_mode<RULE, 2>(mode, units, n, qb, s)
+                    : launch_quantize_mode<RULE, 1>(mode, units, n, qb, s);
 }
 
-cudaError_t launch_quantize(kvq_scale_rule rule, int bpt, int mode, dim3 grid, const QuantBatch& qb, cudaStream_t s)
+cudaError_t launch_quantize(kvq_scale_rule rule, int bpt, int mode, uint64_t units, int n, const QuantBatch& qb,
+                            cudaStream_t s)
 {
     if (rule == KVQ_RULE_STATIC_6)
-        return launch_quantize_bpt<KVQ_RULE_STATIC_6>(bpt, mode, grid, qb, s);
+        return launch_quantize_bpt<KVQ_RULE_STATIC_6>(bpt, mode, units, n, qb, s);
     if (rule == KVQ_RULE_STATIC_4)
-        return launch_quantize_bpt<KVQ_RULE_STATIC_4>(bpt, mode, grid, qb, s);
-    return launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, grid, qb, s);
+        return launch_quantize_bpt<KVQ_RULE_STATIC_4>(bpt, mode, units, n, qb, s);
+    return launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, units, n, qb, s);
 }
 
 kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s,
@@ -558,8 +577,8 @@ kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scal
     if (mode != kYOnly)
         for (int i = 0; i < n; ++i)
             pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
-    const dim3 grid(tiles(pairs ? (qb.n_blocks + 1) / 2 : qb.n_blocks), n);
-    return launched(launch_quantize(rule, pairs ? 2 : 1, mode, grid, qb, s), "quantize_kernel");
+    const uint64_t units = pairs ? (qb.n_blocks + 1) / 2 : qb.n_blocks;
+    return launched(launch_quantize(rule, pairs ? 2 : 1, mode, units, n, qb, s), "quantize_kernel");
 }
 
 // Dequantize blocks [blk_lo, blk_hi) of n equally laid-out tensors; packed/scales point at

@@ -10,16 +10,16 @@
 // Kernels (streaming passes; no tensor cores, no shared-memory staging of data: every
 // access is a fully coalesced 256-bit or narrower vector access):
 //   zero_kernel      clears the amax slots a quantize is about to reduce into.
-//   amax_kernel      max |x| over each tensor: 256-bit loads, per-lane u16x2 max on the
-//                    bf16 bit patterns, warp redux, one atomic max per CTA.
-//   quantize_kernel  one thread per BPT blocks: one 256-bit load per block, block amax,
-//                    e4m3 scale(s) by the rule, e2m1 codes via cvt.satfinite.e2m1x2,
-//                    8 bytes of codes + 1 scale byte per block stored; in its round-trip
-//                    modes it also writes the bf16 reconstruction (fake quantization).
+//   amax_kernel      max |x| over each tensor: 256-bit loads, a max.xorsign.abs.bf16x2
+//                    tree per block, warp redux, one atomic max per CTA.
+//   quantize_kernel  UPT units of BPT blocks per thread: one 256-bit load per block,
+//                    block amax, e4m3 scale(s) by the rule, e2m1 codes via
+//                    cvt.satfinite.e2m1x2, 8 bytes of codes + 1 scale byte per block
+//                    stored; its round-trip modes also write the bf16 reconstruction.
 //   dequant_kernel   the mirror image: 8 bytes + 1 scale byte -> one 256-bit bf16 store
-//                    per block; the cache form looks up each block's chunk amax.
+//                    per block; in a cache, every CTA lies in one chunk (one amax).
 // Every kernel takes a batch of tensors, so one launch covers every layer's K and V of
-// an append or a read.
+// an append or a read, and every launch is a programmatic dependent launch (pdl_begin).
 #include <cuda_runtime.h>
 
 #include <cstdarg>
@@ -507,8 +507,6 @@ kvq_status check_shape(int64_t n_elems, int32_t head_dim)
     return KVQ_OK;
 }
 
-// Quantize a batch of equally sized tensors whose amax slots are given. When
-// compute_amax, the slots are cleared and reduced first.
 // Units per thread of quantize_kernel. The mse rule is instruction-bound; 8 units per
 // thread amortize the per-CTA scale tables (+4% on B200) as long as the launch keeps
 // enough CTAs to fill the GPU many times over (else the last partial wave costs more).
@@ -551,6 +549,8 @@ cudaError_t launch_quantize(kvq_scale_rule rule, int bpt, int mode, uint64_t uni
     return launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, units, n, qb, s);
 }
 
+// Quantize a batch of equally sized tensors whose amax slots are given. When
+// compute_amax, the slots are cleared and reduced first.
 kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s,
                         int mode = kCodes)
 {

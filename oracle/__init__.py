@@ -56,8 +56,10 @@ def _load():
     lib.orc_append.argtypes = [P, P, P, I64, I64, I32, I64, P, I64, I32, I32]
     lib.orc_dequantize_cache.argtypes = [P, P, P, I64, I64, I32, I64, I64, P, I32]
     lib.orc_cache_bytes.argtypes = [I32, I32, I64, I32, I64, P]
+    lib.orc_rtn_quantize.argtypes = [P, I64, I32, I32, P, P]
+    lib.orc_rtn_dequantize.argtypes = [P, P, I64, I32, I32, P]
     for f in ("orc_quantize", "orc_quantize_block_detail", "orc_dequantize", "orc_append",
-              "orc_dequantize_cache", "orc_cache_bytes"):
+              "orc_dequantize_cache", "orc_cache_bytes", "orc_rtn_quantize", "orc_rtn_dequantize"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -184,3 +186,28 @@ def cache_bytes(layers: int, heads: int, capacity_tokens: int, head_dim: int, to
     if rc != 0:
         raise ValueError(f"oracle cache_bytes: status {rc}")
     return int(out[0]), int(out[1]), int(out[2])
+
+
+# ---- RTN integer codecs -----------------------------------------------------------
+
+def rtn_quantize(x_bits: np.ndarray, head_dim: int, bits: int):
+    """Returns (packed uint8[n*bits/8], scales as bf16 bit patterns uint16[n/16])."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1)
+    n = x_bits.size
+    packed = np.zeros(n * bits // 8, np.uint8)
+    scales = np.zeros(n // BLOCK, np.uint16)
+    rc = _load().orc_rtn_quantize(_ptr(x_bits), n, head_dim, bits, _ptr(packed), _ptr(scales))
+    if rc != 0:
+        raise ValueError(f"oracle rtn_quantize: status {rc}")
+    return packed, scales
+
+
+def rtn_dequantize(packed: np.ndarray, scales: np.ndarray, head_dim: int, bits: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16).reshape(-1)
+    n = packed.size * 8 // bits
+    y = np.zeros(n, np.uint16)
+    rc = _load().orc_rtn_dequantize(_ptr(packed), _ptr(scales), n, head_dim, bits, _ptr(y))
+    if rc != 0:
+        raise ValueError(f"oracle rtn_dequantize: status {rc}")
+    return y

@@ -37,6 +37,9 @@
  *   - rule mse keeps R = 4 only when its squared error is strictly smaller than R = 6's.
  *   - the even-indexed element of a pair goes in the low nibble.
  *   - dequant: y = bf16_rne(e2m1_value(q) * S), the product rounded to fp32 first.
+ *
+ * The RTN integer codecs of [STUDY] appendix Table 3 (RTN_INT4, RTN_INT2, and K2_V4 =
+ * INT2 keys with INT4 values) are restated at the end of the file, with their readings.
  */
 #include <math.h>
 #include <pthread.h>
@@ -454,5 +457,89 @@ int orc_cache_bytes(int32_t layers, int32_t heads, int64_t capacity_tokens, int3
     out[0] = tensors * (elems / 2);
     out[1] = tensors * (elems / ORC_BLOCK);
     out[2] = tensors * chunks * 4u;
+    return ORC_OK;
+}
+
+/* ---------------------------------------------------------------- RTN integer codecs */
+
+/* [STUDY] appendix Table 3: "symmetric blockwise quantization ... block_size=16, 2-bit
+ * (4-bit) packed storage plus per-block scales". Readings (listed in the design notes):
+ *   - symmetric levels q in [-qmax, qmax], qmax = 2^(bits-1) - 1 (7 for INT4, 1 for INT2);
+ *   - one 16-bit scale per block, stored as bf16: the study's compression column gives
+ *     5.33x for RTN INT2 = 16 / (2 + 16/16), i.e. 16 scale bits per 16 values;
+ *     S = bf16_rne(amax_b / qmax), the quotient in fp32;
+ *   - q = clamp(round_half_even(x / S), -qmax, qmax), the quotient an IEEE fp32
+ *     division by the stored scale; q = 0 when S == 0;
+ *   - codes are two's complement: INT4 two per byte (even element low nibble), INT2 four
+ *     per byte (element 4j + k in bits 2k..2k+1);
+ *   - dequant: y = bf16_rne(q * S) (the product is exact in fp32). */
+static int rtn_qmax(int bits) { return (1 << (bits - 1)) - 1; }
+
+static void rtn_quantize_block(const uint16_t* xb, int bits, uint8_t* packed_out, uint16_t* scale_out)
+{
+    const int qmax = rtn_qmax(bits);
+    float x[ORC_BLOCK], amax_b = 0.0f;
+    for (int i = 0; i < ORC_BLOCK; ++i) {
+        x[i] = bf16_to_f32(xb[i]);
+        float a = fabsf(x[i]);
+        if (a > amax_b)
+            amax_b = a;
+    }
+    const uint16_t sb = orc_bf16_rne(amax_b / (float)qmax);
+    const float S = bf16_to_f32(sb);
+    int q[ORC_BLOCK];
+    for (int i = 0; i < ORC_BLOCK; ++i) {
+        if (S == 0.0f) {
+            q[i] = 0;
+            continue;
+        }
+        float t = nearbyintf(x[i] / S); /* round half to even (default rounding mode) */
+        if (t > (float)qmax)
+            t = (float)qmax;
+        if (t < -(float)qmax)
+            t = -(float)qmax;
+        q[i] = (int)t;
+    }
+    *scale_out = sb;
+    const int per_byte = 8 / bits, mask = (1 << bits) - 1;
+    for (int j = 0; j < ORC_BLOCK / per_byte; ++j) {
+        int byte = 0;
+        for (int k = 0; k < per_byte; ++k)
+            byte |= (q[per_byte * j + k] & mask) << (bits * k);
+        packed_out[j] = (uint8_t)byte;
+    }
+}
+
+static void rtn_dequantize_block(const uint8_t* packed, uint16_t scale, int bits, uint16_t* y)
+{
+    const float S = bf16_to_f32(scale);
+    const int per_byte = 8 / bits, mask = (1 << bits) - 1;
+    for (int i = 0; i < ORC_BLOCK; ++i) {
+        int v = (packed[i / per_byte] >> (bits * (i % per_byte))) & mask;
+        if (v >= (1 << (bits - 1)))
+            v -= (1 << bits); /* two's complement */
+        y[i] = orc_bf16_rne((float)v * S);
+    }
+}
+
+int orc_rtn_quantize(const uint16_t* x, int64_t n, int32_t head_dim, int32_t bits, uint8_t* packed,
+                     uint16_t* scales)
+{
+    if (check_shape(n, head_dim) != ORC_OK || (bits != 2 && bits != 4))
+        return ORC_ERR_ARG;
+    const int64_t bytes_per_block = ORC_BLOCK * bits / 8;
+    for (int64_t b = 0; b < n / ORC_BLOCK; ++b)
+        rtn_quantize_block(x + b * ORC_BLOCK, bits, packed + b * bytes_per_block, scales + b);
+    return ORC_OK;
+}
+
+int orc_rtn_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t n, int32_t head_dim, int32_t bits,
+                       uint16_t* y)
+{
+    if (check_shape(n, head_dim) != ORC_OK || (bits != 2 && bits != 4))
+        return ORC_ERR_ARG;
+    const int64_t bytes_per_block = ORC_BLOCK * bits / 8;
+    for (int64_t b = 0; b < n / ORC_BLOCK; ++b)
+        rtn_dequantize_block(packed + b * bytes_per_block, scales[b], bits, y + b * ORC_BLOCK);
     return ORC_OK;
 }

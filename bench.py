@@ -13,7 +13,8 @@ sizing, per-chunk amax, block scales, e2m1 packing, and dequantization.
 Other workloads: ``single`` ([4096,128], static_6), ``layer`` (one layer's K and V of
 [1,24,4680,128], mse), ``cache`` (30 layers x {K,V} of [1,24,32760,128]; quantize all,
 dequantize per layer), ``sweep`` ([T,128], --tokens), ``roundtrip`` ([T,128] through the
-fused quantize + dequantize kernel).
+fused quantize + dequantize kernel), ``rtn`` ([T,128] through the RTN INT4 / INT2 codec,
+--bits).
 
 Timing: each bench step is captured as CUDA graphs (one per segment: an append, a
 layer loop of reads, ...), replayed with CUDA events between segments on the launching
@@ -431,7 +432,48 @@ class RoundTrip(Sweep):
         return [self.p[0], self.s[0], self.a[0], self.y[0]]
 
 
-WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip)}
+class Rtn(Sweep):
+    """The RTN integer codec (INT4 / INT2, bf16 scale per 16 values) on [T, 128]:
+    quantize then dequantize."""
+    name = "rtn"
+
+    def __init__(self, args, rank):
+        Sweep.__init__(self, args, rank)
+        self.bits = args.bits
+        self.config["workload"] = f"RTN INT{self.bits} quantize+dequantize: [{self.tokens},128] N(0,1)"
+
+    def setup(self, kvq, inputs, dev):
+        Sweep.setup(self, kvq, inputs, dev)
+        self.p = [torch.empty(self.n * self.bits // 8, dtype=torch.uint8, device=dev)]
+        self.s = [torch.empty(self.n // 16, dtype=torch.bfloat16, device=dev)]
+
+    def segments(self):
+        kvq, bq = self.kvq, 2.0 + self.bits / 8 + 2.0 / 16
+
+        def q():
+            kvq.kvq_rtn_quantize(self.x[0], self.bits, self.D, packed=self.p[0], scales=self.s[0])
+
+        def d():
+            kvq.kvq_rtn_dequantize(self.p[0], self.s[0], self.bits, self.D, y=self.y[0])
+        return [Segment("rtn_quantize", q, 1, self.n * bq, h2d=(self.x[0],)),
+                Segment("rtn_dequantize", d, 1, self.n * bq)]
+
+    def d2h(self):
+        return [self.p[0], self.s[0], self.y[0]]
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        m = min(self.tokens, 1 << 16)
+        xb = inputs.bits(inputs.sweep(self.tokens)[:m])
+        t0, nbytes, reps = time.perf_counter(), 0.0, 0
+        while reps < 1 or time.perf_counter() - t0 < min(budget_s, 5.0):
+            p, s = orc.rtn_quantize(xb, self.D, self.bits)
+            orc.rtn_dequantize(p, s, self.D, self.bits)
+            nbytes += 2 * m * self.D * (2.0 + self.bits / 8 + 2.0 / 16)
+            reps += 1
+        return nbytes, time.perf_counter() - t0, f"first {m} of {self.tokens} rows, {reps} repetitions"
+
+
+WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn)}
 
 
 # ---------------------------------------------------------------------------- runner
@@ -567,6 +609,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="rollout")
     ap.add_argument("--rule", choices=("static_6", "static_4", "mse"), default=None)
     ap.add_argument("--tokens", type=int, default=1 << 24, help="rows of the sweep workload")
+    ap.add_argument("--bits", type=int, choices=(2, 4), default=4, help="bits of the rtn workload")
     ap.add_argument("--small", action="store_true", help="a reduced shape of the workload (for tests)")
     ap.add_argument("--no-graphs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -628,7 +671,8 @@ def main():
     dom_ms = kind_ms[dom] / args.steps
     achieved = kind_bytes[dom] / (dom_ms * 1e-3) / 1e9
     per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
-                "roundtrip": B_AMAX + B_QUANT + 2.0}[dom]
+                "roundtrip": B_AMAX + B_QUANT + 2.0,
+                "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16, "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}[dom]
     tb = measured_traffic(dom)
     elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -207,6 +207,39 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
                                       int64_t row_begin, int64_t row_end, kvq_stream_t stream);
 
 /*
+ * RTN integer codecs: the RTN_INT4 / RTN_INT2 rows of "KV Cache Quantization for
+ * Self-Forcing Video Generation: A 33-Method Empirical Study", appendix Table 3
+ * (symmetric blockwise quantization of K and V, block_size=16, 4-bit / 2-bit packed
+ * storage plus per-block scales); RTN_K2_V4 is bits = 2 for K and 4 for V. Per block of
+ * 16 elements, qmax = 2^(bits-1) - 1:
+ *     S = bf16_rne(amax_b / qmax)            one bf16 scale per block (16 bits per 16
+ *                                            values: the study's 5.33x for INT2)
+ *     q = round_half_even(x / S) in [-qmax, qmax], 0 when S == 0 (IEEE fp32 quotient)
+ *     y = bf16_rne(q * S)
+ * Codes are two's complement; INT4 two per byte (even element in the low nibble), INT2
+ * four per byte (element 4j + k in bits 2k..2k+1). There is no global scale. A cache
+ * append or range read is the same call on pointers offset into the cache buffers.
+ *
+ * kvq_rtn_quantize
+ *   x        device, bf16[n_elems], 32-byte aligned (n_elems a multiple of head_dim).
+ *   bits     2 or 4.
+ *   packed   device, uint8[n_elems * bits / 8], 2*bits-byte aligned. Written.
+ *   scales   device, bf16 bit patterns uint16[n_elems / 16], 2-byte aligned. Written.
+ * kvq_rtn_dequantize -- the inverse; y device bf16[n_elems], 32-byte aligned. Written.
+ * The _batch forms take host arrays of n_tensors device pointers of one size and bits.
+ */
+kvq_status kvq_rtn_quantize(const void* x, int64_t n_elems, int32_t head_dim, int32_t bits, uint8_t* packed,
+                            uint16_t* scales, kvq_stream_t stream);
+kvq_status kvq_rtn_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t n_elems, int32_t head_dim,
+                              int32_t bits, void* y, kvq_stream_t stream);
+kvq_status kvq_rtn_quantize_batch(const void* const* xs, int32_t n_tensors, int64_t n_elems, int32_t head_dim,
+                                  int32_t bits, uint8_t* const* packed, uint16_t* const* scales,
+                                  kvq_stream_t stream);
+kvq_status kvq_rtn_dequantize_batch(const uint8_t* const* packed, const uint16_t* const* scales, int32_t n_tensors,
+                                    int64_t n_elems, int32_t head_dim, int32_t bits, void* const* ys,
+                                    kvq_stream_t stream);
+
+/*
  * kvq_cache_bytes -- host only. Bytes of a cache of `layers` layers x {K, V}, each
  *   capacity_tokens x heads rows of head_dim, chunks of tokens_per_chunk tokens:
  *     packed = 2*layers * capacity_tokens*heads*head_dim / 2

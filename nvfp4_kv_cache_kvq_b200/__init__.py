@@ -58,6 +58,10 @@ def load() -> ctypes.CDLL:
                                  ctypes.POINTER(P), P],
         "kvq_quantize_dequantize": [P, I64, I32, I32, P, P, P, P, P, P],
         "kvq_dequantize": [P, P, P, I64, I32, P, P],
+        "kvq_rtn_quantize": [P, I64, I32, I32, P, P, P],
+        "kvq_rtn_dequantize": [P, P, I64, I32, I32, P, P],
+        "kvq_rtn_quantize_batch": [ctypes.POINTER(P), I32, I64, I32, I32, ctypes.POINTER(P), ctypes.POINTER(P), P],
+        "kvq_rtn_dequantize_batch": [ctypes.POINTER(P), ctypes.POINTER(P), I32, I64, I32, I32, ctypes.POINTER(P), P],
         "kvq_append": [CP, I64, P, I64, I32, P],
         "kvq_append_batch": [CP, ctypes.POINTER(I64), ctypes.POINTER(P), I32, I64, I32, P],
         "kvq_dequantize_cache": [CP, I64, I64, P, P],
@@ -208,6 +212,54 @@ def kvq_quantize_dequantize(x: torch.Tensor, head_dim: int | None = None, rule="
                                           None if scales is None else _dev(scales, "scales"), _dev(y, "y"),
                                           _stream(stream, dev)))
     return y, packed, scales, (amax_out if amax_out is not None else amax_in)
+
+
+def kvq_rtn_quantize(x: torch.Tensor, bits: int, head_dim: int | None = None, packed: torch.Tensor | None = None,
+                     scales: torch.Tensor | None = None, stream=None):
+    """RTN INT4 / INT2 of a bf16 tensor. Returns (packed uint8[n*bits/8], scales bf16[n/16])."""
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    n, dev = x.numel(), x.device
+    head_dim = int(head_dim or x.shape[-1])
+    packed = packed if packed is not None else torch.empty(n * bits // 8, dtype=torch.uint8, device=dev)
+    scales = scales if scales is not None else torch.empty(n // BLOCK, dtype=torch.bfloat16, device=dev)
+    _check(load().kvq_rtn_quantize(_dev(x, "x"), n, head_dim, int(bits), _dev(packed, "packed"),
+                                   _dev(scales, "scales"), _stream(stream, dev)))
+    return packed, scales
+
+
+def kvq_rtn_dequantize(packed: torch.Tensor, scales: torch.Tensor, bits: int, head_dim: int,
+                       y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    n = packed.numel() * 8 // int(bits)
+    dev = packed.device
+    y = y if y is not None else torch.empty(n, dtype=torch.bfloat16, device=dev)
+    _check(load().kvq_rtn_dequantize(_dev(packed, "packed"), _dev(scales, "scales"), n, int(head_dim), int(bits),
+                                     _dev(y, "y"), _stream(stream, dev)))
+    return y
+
+
+def kvq_rtn_quantize_batch(xs, bits: int, head_dim: int | None = None, packed=None, scales=None, stream=None):
+    n = len(xs)
+    if n == 0:
+        return [], []
+    numel, dev = xs[0].numel(), xs[0].device
+    head_dim = int(head_dim or xs[0].shape[-1])
+    packed = packed or [torch.empty(numel * bits // 8, dtype=torch.uint8, device=dev) for _ in xs]
+    scales = scales or [torch.empty(numel // BLOCK, dtype=torch.bfloat16, device=dev) for _ in xs]
+    _check(load().kvq_rtn_quantize_batch(_ptrs(xs, "x"), n, numel, head_dim, int(bits), _ptrs(packed, "packed"),
+                                         _ptrs(scales, "scales"), _stream(stream, dev)))
+    return packed, scales
+
+
+def kvq_rtn_dequantize_batch(packed, scales, bits: int, head_dim: int, ys=None, stream=None):
+    n = len(packed)
+    if n == 0:
+        return []
+    numel, dev = packed[0].numel() * 8 // int(bits), packed[0].device
+    ys = ys or [torch.empty(numel, dtype=torch.bfloat16, device=dev) for _ in packed]
+    _check(load().kvq_rtn_dequantize_batch(_ptrs(packed, "packed"), _ptrs(scales, "scales"), n, numel,
+                                           int(head_dim), int(bits), _ptrs(ys, "y"), _stream(stream, dev)))
+    return ys
 
 
 class KVCache:

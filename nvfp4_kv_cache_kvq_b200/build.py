@@ -7,8 +7,9 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", "kvq.cu")]
-DEPS = SOURCES + [os.path.join(PKG, "csrc", "kvq_device.cuh"), os.path.join(ROOT, "include", "kvq.h")]
+SOURCES = [os.path.join(PKG, "csrc", "kvq.cu"), os.path.join(PKG, "csrc", "kvq_rtn.cu")]
+DEPS = SOURCES + [os.path.join(PKG, "csrc", "kvq_device.cuh"), os.path.join(PKG, "csrc", "kvq_common.h"),
+                  os.path.join(ROOT, "include", "kvq.h")]
 LIB = os.path.join(PKG, "_build", "libkvq.so")
 
 NVCC_FLAGS = [

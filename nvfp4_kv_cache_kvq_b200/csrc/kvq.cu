@@ -688,6 +688,7 @@ kvq_status kvq_quantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_sc
                         const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
                         kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_quantize");
     return quantize_impl("kvq_quantize", &x, 1, n_elems, head_dim, rule, amax_in ? &amax_in : nullptr,
                          amax_out ? &amax_out : nullptr, &packed, &scales, nullptr, kCodes,
                          reinterpret_cast<cudaStream_t>(stream));
@@ -697,6 +698,7 @@ kvq_status kvq_quantize_batch(const void* const* xs, int32_t n_tensors, int64_t 
                               kvq_scale_rule rule, const float* const* amax_in, float* const* amax_out,
                               uint8_t* const* packed, uint8_t* const* scales, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_quantize_batch");
     return quantize_impl("kvq_quantize_batch", xs, n_tensors, n_elems, head_dim, rule, amax_in, amax_out, packed,
                          scales, nullptr, kCodes, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -705,6 +707,7 @@ kvq_status kvq_quantize_dequantize(const void* x, int64_t n_elems, int32_t head_
                                    const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
                                    void* y, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_quantize_dequantize");
     if ((packed == nullptr) != (scales == nullptr))
         return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize_dequantize: packed and scales must be both given or both null");
     const int mode = packed ? kCodesAndY : kYOnly;
@@ -717,6 +720,7 @@ kvq_status kvq_dequantize_batch(const uint8_t* const* packed, const uint8_t* con
                                 int32_t n_tensors, int64_t n_elems, int32_t head_dim, void* const* ys,
                                 kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_dequantize_batch");
     return dequantize_impl(packed, scales, amax, n_tensors, n_elems, head_dim, ys,
                            reinterpret_cast<cudaStream_t>(stream));
 }
@@ -724,12 +728,14 @@ kvq_status kvq_dequantize_batch(const uint8_t* const* packed, const uint8_t* con
 kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const float* amax, int64_t n_elems,
                           int32_t head_dim, void* y, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_dequantize");
     return dequantize_impl(&packed, &scales, &amax, 1, n_elems, head_dim, &y, reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_append_batch(const kvq_cache* caches, const int64_t* row_offsets, const void* const* xs,
                             int32_t n_tensors, int64_t n_rows, kvq_scale_rule rule, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_append_batch");
     kvq_status st;
     if ((st = check_rule(rule)) != KVQ_OK)
         return st;
@@ -789,12 +795,14 @@ kvq_status kvq_append_batch(const kvq_cache* caches, const int64_t* row_offsets,
 kvq_status kvq_append(const kvq_cache* cache, int64_t row_offset, const void* x, int64_t n_rows,
                       kvq_scale_rule rule, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_append");
     return kvq_append_batch(cache, &row_offset, &x, 1, n_rows, rule, stream);
 }
 
 kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, int32_t n_tensors,
                                       int64_t row_begin, int64_t row_end, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_dequantize_cache_batch");
     kvq_status st;
     if (n_tensors < 0)
         return fail(KVQ_ERR_INVALID_ARG, "kvq_dequantize_cache_batch: negative count");
@@ -847,6 +855,7 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
 kvq_status kvq_dequantize_cache(const kvq_cache* cache, int64_t row_begin, int64_t row_end, void* y,
                                 kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_dequantize_cache");
     return kvq_dequantize_cache_batch(cache, &y, 1, row_begin, row_end, stream);
 }
 
@@ -854,6 +863,7 @@ kvq_status kvq_cache_bytes(int32_t layers, int32_t heads, int64_t capacity_token
                            int64_t tokens_per_chunk, uint64_t* packed_bytes, uint64_t* scale_bytes,
                            uint64_t* amax_bytes)
 {
+    NvtxRange nvtx_range("kvq_cache_bytes");
     if (layers <= 0 || heads <= 0 || capacity_tokens < 0 || head_dim <= 0 || head_dim % kBlock != 0 ||
         tokens_per_chunk <= 0)
         return fail(KVQ_ERR_INVALID_ARG, "kvq_cache_bytes: bad dimensions");

@@ -8,9 +8,20 @@
 #include <cstdint>
 #include <cstdio>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "kvq.h"
 
 namespace kvq {
+
+// An NVTX range around each entry point, so profilers show the library's calls by name
+// (free when no tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kBlock = 16;  // elements per quantization block
 constexpr int kThreads = 256;

@@ -220,12 +220,14 @@ extern "C" {
 kvq_status kvq_rtn_quantize(const void* x, int64_t n_elems, int32_t head_dim, int32_t bits, uint8_t* packed,
                             uint16_t* scales, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_rtn_quantize");
     return rtn_impl(true, &x, &packed, &scales, 1, n_elems, head_dim, bits, reinterpret_cast<cudaStream_t>(stream));
 }
 
 kvq_status kvq_rtn_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t n_elems, int32_t head_dim,
                               int32_t bits, void* y, kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_rtn_dequantize");
     const void* yy = y;
     uint8_t* p = const_cast<uint8_t*>(packed);
     uint16_t* sc = const_cast<uint16_t*>(scales);
@@ -236,6 +238,7 @@ kvq_status kvq_rtn_quantize_batch(const void* const* xs, int32_t n_tensors, int6
                                   int32_t bits, uint8_t* const* packed, uint16_t* const* scales,
                                   kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_rtn_quantize_batch");
     return rtn_impl(true, xs, packed, scales, n_tensors, n_elems, head_dim, bits,
                     reinterpret_cast<cudaStream_t>(stream));
 }
@@ -244,6 +247,7 @@ kvq_status kvq_rtn_dequantize_batch(const uint8_t* const* packed, const uint16_t
                                     int64_t n_elems, int32_t head_dim, int32_t bits, void* const* ys,
                                     kvq_stream_t stream)
 {
+    NvtxRange nvtx_range("kvq_rtn_dequantize_batch");
     return rtn_impl(false, const_cast<const void* const*>(ys), const_cast<uint8_t* const*>(packed),
                     const_cast<uint16_t* const*>(scales), n_tensors, n_elems, head_dim, bits,
                     reinterpret_cast<cudaStream_t>(stream));

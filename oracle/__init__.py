@@ -58,8 +58,11 @@ def _load():
     lib.orc_cache_bytes.argtypes = [I32, I32, I64, I32, I64, P]
     lib.orc_rtn_quantize.argtypes = [P, I64, I32, I32, P, P]
     lib.orc_rtn_dequantize.argtypes = [P, P, I64, I32, I32, P]
+    lib.orc_scales_to_blocked.argtypes = [P, I64, I32, P]
+    lib.orc_scales_from_blocked.argtypes = [P, I64, I32, P]
     for f in ("orc_quantize", "orc_quantize_block_detail", "orc_dequantize", "orc_append",
-              "orc_dequantize_cache", "orc_cache_bytes", "orc_rtn_quantize", "orc_rtn_dequantize"):
+              "orc_dequantize_cache", "orc_cache_bytes", "orc_rtn_quantize", "orc_rtn_dequantize",
+              "orc_scales_to_blocked", "orc_scales_from_blocked"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -211,3 +214,25 @@ def rtn_dequantize(packed: np.ndarray, scales: np.ndarray, head_dim: int, bits: 
     if rc != 0:
         raise ValueError(f"oracle rtn_dequantize: status {rc}")
     return y
+
+
+# ---- blocked scale layout ----------------------------------------------------------
+
+def blocked_bytes(rows: int, cols: int) -> int:
+    return -(-rows // 128) * 128 * -(-cols // 4) * 4
+
+
+def scales_to_blocked(scales: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    scales = np.ascontiguousarray(scales, dtype=np.uint8).reshape(-1)
+    out = np.zeros(blocked_bytes(rows, cols), np.uint8)
+    if _load().orc_scales_to_blocked(_ptr(scales), rows, cols, _ptr(out)) != 0:
+        raise ValueError("oracle scales_to_blocked: bad shape")
+    return out
+
+
+def scales_from_blocked(blocked: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    blocked = np.ascontiguousarray(blocked, dtype=np.uint8).reshape(-1)
+    out = np.zeros(rows * cols, np.uint8)
+    if _load().orc_scales_from_blocked(_ptr(blocked), rows, cols, _ptr(out)) != 0:
+        raise ValueError("oracle scales_from_blocked: bad shape")
+    return out

@@ -543,3 +543,38 @@ int orc_rtn_dequantize(const uint8_t* packed, const uint16_t* scales, int64_t n,
         rtn_dequantize_block(packed + b * bytes_per_block, scales[b], bits, y + b * ORC_BLOCK);
     return ORC_OK;
 }
+
+/* ---------------------------------------------------------------- blocked scale layout */
+
+/* The "blocked" layout of a [rows, cols] scale matrix that block-scaled MMA operands use
+ * and that [NVFP4] "Stage 3" step 1 undoes ("from_blocked"): rows padded to a multiple
+ * of 128, cols to a multiple of 4, zero filled; 128 x 4 tiles of 512 bytes in row-tile
+ * major order; inside a tile, scale (r, c) at byte (r % 32) * 16 + ((r % 128) / 32) * 4
+ * + c % 4. */
+static int64_t blocked_offset(int64_t r, int64_t c, int64_t col_tiles)
+{
+    return ((r / 128) * col_tiles + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+int orc_scales_to_blocked(const uint8_t* scales, int64_t rows, int32_t cols, uint8_t* blocked)
+{
+    if (rows < 0 || cols <= 0)
+        return ORC_ERR_ARG;
+    const int64_t row_tiles = (rows + 127) / 128, col_tiles = (cols + 3) / 4;
+    memset(blocked, 0, (size_t)(row_tiles * col_tiles * 512));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            blocked[blocked_offset(r, c, col_tiles)] = scales[r * cols + c];
+    return ORC_OK;
+}
+
+int orc_scales_from_blocked(const uint8_t* blocked, int64_t rows, int32_t cols, uint8_t* scales)
+{
+    if (rows < 0 || cols <= 0)
+        return ORC_ERR_ARG;
+    const int64_t col_tiles = (cols + 3) / 4;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c)
+            scales[r * cols + c] = blocked[blocked_offset(r, c, col_tiles)];
+    return ORC_OK;
+}

@@ -240,6 +240,26 @@ kvq_status kvq_rtn_dequantize_batch(const uint8_t* const* packed, const uint16_t
                                     kvq_stream_t stream);
 
 /*
+ * Blocked scale layout: the 128 x 4 tiles block-scaled MMA operands read ("How NVFP4
+ * Quantization Works in LongLive 2.0", "Stage 3", step 1: the dequantizer first undoes
+ * it, "from_blocked"). A [rows, cols] matrix of one-byte scales (row-major: the scales
+ * array of kvq_quantize for a rows x head_dim tensor, cols = head_dim / 16) is padded
+ * with zeros to rows' = ceil(rows/128)*128 and cols' = ceil(cols/4)*4 and cut into
+ * 128 x 4 tiles of 512 bytes, in row-tile-major order; inside a tile, scale (r, c) sits
+ * at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
+ *
+ * kvq_scales_to_blocked    scales (device, rows*cols bytes) -> blocked (device,
+ *                          kvq_blocked_scale_bytes bytes, 4-byte aligned, padding zeroed).
+ * kvq_scales_from_blocked  the inverse; writes rows*cols bytes.
+ * kvq_blocked_scale_bytes  host only: rows' * cols'.
+ */
+kvq_status kvq_scales_to_blocked(const uint8_t* scales, int64_t rows, int32_t cols, uint8_t* blocked,
+                                 kvq_stream_t stream);
+kvq_status kvq_scales_from_blocked(const uint8_t* blocked, int64_t rows, int32_t cols, uint8_t* scales,
+                                   kvq_stream_t stream);
+kvq_status kvq_blocked_scale_bytes(int64_t rows, int32_t cols, uint64_t* bytes);
+
+/*
  * kvq_cache_bytes -- host only. Bytes of a cache of `layers` layers x {K, V}, each
  *   capacity_tokens x heads rows of head_dim, chunks of tokens_per_chunk tokens:
  *     packed = 2*layers * capacity_tokens*heads*head_dim / 2

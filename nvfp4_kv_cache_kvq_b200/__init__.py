@@ -67,6 +67,9 @@ def load() -> ctypes.CDLL:
         "kvq_dequantize_cache": [CP, I64, I64, P, P],
         "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
         "kvq_cache_bytes": [I32, I32, I64, I32, I64, U64P, U64P, U64P],
+        "kvq_scales_to_blocked": [P, I64, I32, P, P],
+        "kvq_scales_from_blocked": [P, I64, I32, P, P],
+        "kvq_blocked_scale_bytes": [I64, I32, U64P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -352,6 +355,31 @@ def kvq_cache_bytes(layers: int, heads: int, capacity_tokens: int, head_dim: int
     _check(load().kvq_cache_bytes(int(layers), int(heads), int(capacity_tokens), int(head_dim),
                                   int(tokens_per_chunk), ctypes.byref(p), ctypes.byref(s), ctypes.byref(a)))
     return p.value, s.value, a.value
+
+
+def kvq_blocked_scale_bytes(rows: int, cols: int) -> int:
+    b = ctypes.c_uint64()
+    _check(load().kvq_blocked_scale_bytes(int(rows), int(cols), ctypes.byref(b)))
+    return b.value
+
+
+def kvq_scales_to_blocked(scales: torch.Tensor, rows: int, cols: int, blocked: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    """Row-major [rows, cols] one-byte scales -> the blocked 128 x 4 tile layout."""
+    if blocked is None:
+        blocked = torch.empty(kvq_blocked_scale_bytes(rows, cols), dtype=torch.uint8, device=scales.device)
+    _check(load().kvq_scales_to_blocked(_dev(scales, "scales"), int(rows), int(cols), _dev(blocked, "blocked"),
+                                        _stream(stream, scales.device)))
+    return blocked
+
+
+def kvq_scales_from_blocked(blocked: torch.Tensor, rows: int, cols: int, scales: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
+    if scales is None:
+        scales = torch.empty(rows * cols, dtype=torch.uint8, device=blocked.device)
+    _check(load().kvq_scales_from_blocked(_dev(blocked, "blocked"), int(rows), int(cols), _dev(scales, "scales"),
+                                          _stream(stream, blocked.device)))
+    return scales
 
 
 def loaded_library() -> str | None:

@@ -583,13 +583,29 @@ def capture(segs, use_graphs):
 
 def run_step(segs, events, e2e=None):
     """One bench step on the current stream; events[i] is recorded before segment i and
-    events[-1] after the last. With e2e, every segment's inputs are first copied in
-    from pinned host memory (inside its event interval)."""
+    events[-1] after the last. With e2e, every segment's inputs are copied in from pinned
+    host memory on a copy stream that starts with the step and runs ahead of the compute
+    (each segment waits only for its own inputs), and the step's outputs are copied back
+    at the end, all inside the timed interval."""
+    main = torch.cuda.current_stream()
+    events[0].record()
+    ready = [None] * len(segs)
+    if e2e is not None:
+        cs = e2e["stream"]
+        cs.wait_event(events[0])
+        with torch.cuda.stream(cs):
+            for i, seg in enumerate(segs):
+                if seg.h2d is None:
+                    continue
+                for dst, src in zip(seg.h2d, e2e["h2d"][i]):
+                    dst.copy_(src, non_blocking=True)
+                ready[i] = torch.cuda.Event()
+                ready[i].record(cs)
     for i, seg in enumerate(segs):
-        events[i].record()
-        if e2e is not None and seg.h2d is not None:
-            for dst, src in zip(seg.h2d, e2e["h2d"][i]):
-                dst.copy_(src, non_blocking=True)
+        if i > 0:
+            events[i].record()
+        if ready[i] is not None:
+            main.wait_event(ready[i])
         if seg.graph is not None:
             seg.graph.replay()
         else:
@@ -706,8 +722,9 @@ def main():
 
 
 def run_e2e(args, wl, segs, bytes_step, world):
-    """The same steps with every segment's inputs copied in from pinned host memory and
-    the step's outputs copied back, inside the timed region."""
+    """The same steps with every segment's inputs copied in from pinned host memory (on a
+    copy stream overlapping the compute) and the step's outputs copied back, inside the
+    timed region."""
     h2d, h2d_bytes = [], 0
     for seg in segs:
         if seg.h2d is None:
@@ -723,7 +740,7 @@ def run_e2e(args, wl, segs, bytes_step, world):
     d2h_src = wl.d2h()
     d2h_dst = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d2h_src]
     d2h_bytes = sum(t.numel() * t.element_size() for t in d2h_src)
-    e2e = {"h2d": h2d, "d2h_src": d2h_src, "d2h_dst": d2h_dst}
+    e2e = {"h2d": h2d, "d2h_src": d2h_src, "d2h_dst": d2h_dst, "stream": torch.cuda.Stream()}
     events = [torch.cuda.Event(enable_timing=True) for _ in range(len(segs) + 1)]
     run_step(segs, events, e2e)
     torch.cuda.synchronize()

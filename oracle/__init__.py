@@ -236,3 +236,25 @@ def scales_from_blocked(blocked: np.ndarray, rows: int, cols: int) -> np.ndarray
     if _load().orc_scales_from_blocked(_ptr(blocked), rows, cols, _ptr(out)) != 0:
         raise ValueError("oracle scales_from_blocked: bad shape")
     return out
+
+
+# ---- attention over a dequantized cache ---------------------------------------------
+
+def attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, n_queries: int, n_keys: int,
+              heads: int, head_dim: int, scale: float) -> np.ndarray:
+    """softmax(Q K^T * scale) V per head, in fp64, on bf16 inputs given as bit patterns:
+    q [n_queries, heads, head_dim], k and v [n_keys, heads, head_dim] (token-major, the
+    cache's row order). Returns fp64 [n_queries, heads, head_dim]. This is the consumer
+    the pages place after dequantization ("dequantize the active cache back to dense
+    BF16 before attention", Self-Forcing study, appendix Table 3)."""
+    def f64(b, rows):
+        u = (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+        return u.astype(np.float64).reshape(rows, heads, head_dim)
+    q, k, v = f64(q_bits, n_queries), f64(k_bits, n_keys), f64(v_bits, n_keys)
+    out = np.empty((n_queries, heads, head_dim))
+    for h in range(heads):
+        s = q[:, h, :] @ k[:, h, :].T * scale
+        s -= s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        out[:, h, :] = (p @ v[:, h, :]) / p.sum(axis=1, keepdims=True)
+    return out

@@ -52,7 +52,8 @@ def kernel_source_sha256() -> str:
     import hashlib
 
     h = hashlib.sha256()
-    for rel in ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh"):
+    for rel in ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_rtn.cu",
+                "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh", "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -70,6 +71,14 @@ def measured_traffic(kind: str):
         return None
     k = t.get("kernels", {}).get(kind)
     return None if k is None else float(k["dram_bytes_per_elem"])
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (MEASURED_PEAKS.json bf16_tflops_sustained)"
+    except Exception:
+        return 1400.0, "fallback (sustained dense bf16)"
 
 
 def peaks():
@@ -473,7 +482,119 @@ class Rtn(Sweep):
         return nbytes, time.perf_counter() - t0, f"first {m} of {self.tokens} rows, {reps} repetitions"
 
 
-WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn)}
+class Attention:
+    """The rollout's attention at its last frame, reading the packed cache directly: for
+    every layer, one frame of 1560 queries x 12 heads attends to that layer's 60-frame
+    K/V cache (93,600 tokens) through kvq_attention. The same work done unfused --
+    kvq_dequantize_cache_batch into bf16 buffers, then torch's scaled_dot_product_attention
+    -- is timed beside it (``unfused``), with the bf16 bytes it has to hold."""
+    name = "attention"
+
+    def __init__(self, args, rank):
+        self.layers, self.heads, self.tokens, self.frames, self.D = 30, 12, 1560, 60, 128
+        if args.small:
+            self.layers, self.heads, self.tokens, self.frames = 2, 2, 120, 6
+        self.rule = args.rule or "mse"
+        self.rank = rank
+        self.rpc = self.tokens * self.heads
+        self.n_keys = self.tokens * self.frames
+        self.flops_layer = 4.0 * self.tokens * self.n_keys * self.heads * self.D
+        # packed K and V (codes + scales) read once, queries read, output written
+        self.bytes_layer = 2 * self.n_keys * self.heads * self.D * 0.5625 + 2 * self.rpc * self.D * 2.0
+        self.config = {
+            "workload": f"fused NVFP4-cache attention: {self.layers} layers, {self.tokens} queries x {self.heads} "
+                        f"heads over a {self.frames}-frame cache ({self.n_keys} tokens), head_dim {self.D}, "
+                        f"Student-t(4) K/V appended with rule {self.rule}, N(0,1) queries",
+            "model": "Wan-shaped self-forcing KV cache (synthetic)", "global_batch": 1, "seq_len": self.n_keys,
+            "parallelism": "replica per GPU", "l2": "inputs larger than L2 (each layer's packed cache is 162 MB)",
+        }
+
+    def setup(self, kvq, inputs, dev):
+        T = 2 * self.layers
+        self.caches = kvq.allocate_caches(self.layers, self.heads, self.n_keys, self.D, self.tokens, dev)
+        for f in range(self.frames):
+            xs = [inputs.rollout_chunk(f + self.frames * self.rank, t, heads=self.heads, tokens=self.tokens,
+                                       device=dev) for t in range(T)]
+            kvq.kvq_append_batch(self.caches, [f * self.rpc] * T, xs, self.rule)
+        self.q = torch.stack([inputs.queries(l + self.layers * self.rank, heads=self.heads, tokens=self.tokens,
+                                             device=dev) for l in range(self.layers)])
+        self.o = torch.empty_like(self.q)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.kvq = kvq
+        torch.cuda.synchronize()
+
+    def segments(self):
+        kvq = self.kvq
+
+        def attn():
+            for l in range(self.layers):
+                kvq.kvq_attention(self.q[l], self.caches[2 * l], self.caches[2 * l + 1], self.n_keys,
+                                  out=self.o[l], status=self.status)
+        seg = Segment("attention", attn, self.layers, self.layers * self.bytes_layer, h2d=(self.q,))
+        seg.flops = self.layers * self.flops_layer
+        return [seg]
+
+    def d2h(self):
+        return [self.o]
+
+    def tokens_per_step(self):
+        return self.tokens * self.layers
+
+    def check(self):
+        if int(self.status.item()) != 0:
+            raise RuntimeError("kvq_attention reported an on-chip wait timeout")
+
+    def unfused(self, steps):
+        """Dequantize each layer's K and V to bf16, then torch's SDPA, timed with events."""
+        import torch.nn.functional as F
+
+        kvq, H, D = self.kvq, self.heads, self.D
+        rows = self.n_keys * H
+        yk = torch.empty(rows * D, dtype=torch.bfloat16, device=self.q.device)
+        yv = torch.empty_like(yk)
+
+        def layer(l):
+            kvq.kvq_dequantize_cache_batch(self.caches[2 * l:2 * l + 2], 0, rows, [yk, yv])
+            k = yk.view(1, self.n_keys, H, D).transpose(1, 2)
+            v = yv.view(1, self.n_keys, H, D).transpose(1, 2)
+            q = self.q[l].unsqueeze(0).transpose(1, 2)
+            return F.scaled_dot_product_attention(q, k, v).transpose(1, 2)
+
+        for l in range(self.layers):
+            out = layer(l)
+        torch.cuda.synchronize()
+        diff = float((out[0].float() - self.o[self.layers - 1].float()).abs().max())
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ms = []
+        for _ in range(steps):
+            e0.record()
+            for l in range(self.layers):
+                layer(l)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return {"ms_per_step": sum(ms) / len(ms), "what": "kvq_dequantize_cache_batch + torch SDPA per layer",
+                "transient_bf16_bytes": 2 * rows * D * 2, "max_abs_diff_vs_fused": diff}
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        """Layer 0: the oracle appends the cache (untimed), then dequantizes K and V and
+        computes a few query rows' attention in fp64 (timed); the bytes are the layer's
+        algorithmic bytes scaled by the share of query rows done."""
+        caches = [orc.Cache(self.frames * self.rpc, self.rpc, self.D) for _ in range(2)]
+        for f in range(self.frames):
+            for t in range(2):
+                caches[t].append(f * self.rpc, inputs.bits(inputs.rollout_chunk(f, t, heads=self.heads,
+                                                                                tokens=self.tokens)), self.rule)
+        qb = inputs.bits(inputs.queries(0, heads=self.heads, tokens=self.tokens)).reshape(self.tokens, -1)
+        m = 4
+        t0 = time.perf_counter()
+        kb, vb = caches[0].dequantize(0, self.n_keys * self.heads), caches[1].dequantize(0, self.n_keys * self.heads)
+        orc.attention(qb[:m].reshape(-1), kb, vb, m, self.n_keys, self.heads, self.D, self.D ** -0.5)
+        dt = time.perf_counter() - t0
+        return self.bytes_layer * m / self.tokens, dt, f"layer 0, {m} of {self.tokens} query rows"
+
+
+WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention)}
 
 
 # ---------------------------------------------------------------------------- runner
@@ -686,16 +807,27 @@ def main():
     dom = max(kinds, key=lambda k: kind_ms[k])
     dom_ms = kind_ms[dom] / args.steps
     achieved = kind_bytes[dom] / (dom_ms * 1e-3) / 1e9
-    per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
-                "roundtrip": B_AMAX + B_QUANT + 2.0,
-                "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16, "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}[dom]
-    tb = measured_traffic(dom)
-    elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom]
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
-                "traffic": None if tb is None else tb * elems_per_launch,
-                "alg_bytes_per_launch": kind_bytes[dom] / kind_launch[dom],
-                "launches_per_step": kind_launch[dom], "ms_per_step": dom_ms}
+    dom_flops = sum(getattr(s, "flops", 0.0) for s in segs if s.kind == dom)
+    if dom_flops:
+        # a contraction: against the measured dense bf16 GEMM peak (sustained: the kernel
+        # runs back to back for the whole timed region)
+        tflops = dom_flops / (dom_ms * 1e-3) / 1e12
+        tpeak, tsrc = tensor_peak()
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": tflops / tpeak, "peak_source": tsrc, "traffic": None,
+                    "flops_per_launch": dom_flops / kind_launch[dom], "launches_per_step": kind_launch[dom],
+                    "ms_per_step": dom_ms, "hbm_GB_s": achieved}
+    else:
+        per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
+                    "roundtrip": B_AMAX + B_QUANT + 2.0, "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16,
+                    "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}[dom]
+        tb = measured_traffic(dom)
+        elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom]
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
+                    "traffic": None if tb is None else tb * elems_per_launch,
+                    "alg_bytes_per_launch": kind_bytes[dom] / kind_launch[dom],
+                    "launches_per_step": kind_launch[dom], "ms_per_step": dom_ms}
     per_kind = {k: {"ms_per_step": kind_ms[k] / args.steps,
                     "GB_s": kind_bytes[k] / (kind_ms[k] / args.steps * 1e-3) / 1e9 if kind_ms[k] else None,
                     "launches_per_step": kind_launch[k]} for k in kinds}
@@ -707,6 +839,10 @@ def main():
             "roofline": roofline, "kernels": per_kind, "gpu_launches": sum(s.launches for s in segs) * args.steps,
             "clocks": sampler.summary(), "graphs": not args.no_graphs}
 
+    if hasattr(wl, "check"):
+        wl.check()
+    if hasattr(wl, "unfused"):
+        line["unfused"] = wl.unfused(args.steps)
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, wl, segs, bytes_step, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -207,6 +207,30 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
                                       int64_t row_begin, int64_t row_end, kvq_stream_t stream);
 
 /*
+ * kvq_attention -- softmax attention out = softmax(softmax_scale * Q K^T) V per head,
+ *   reading K and V straight from their NVFP4 caches: each tile of keys is dequantized
+ *   in on-chip memory to the same bf16 values kvq_dequantize_cache writes, so no dense
+ *   bf16 copy of the cache is ever stored ("How to Use KV Cache Quantization with
+ *   LongLive's LongLiveQuantizationConfig", "CUDA De-quantization Pipeline": dequantize
+ *   during the attention operation; Self-Forcing study, abstract and Figure 6: the
+ *   transient BF16 buffers of dequantize-then-attend set the peak memory). Every query
+ *   attends to cache tokens [0, n_keys) (no mask); P is rounded to bf16 before P V and
+ *   both products accumulate in fp32 on the tensor cores.
+ *   q            device, bf16[n_queries, heads, 128] (token-major), 16-byte aligned.
+ *   k_cache,     host pointers to the K and V cache views: rows are token * heads + head,
+ *   v_cache      head_dim 128, rows_per_chunk a multiple of heads and equal in both,
+ *                n_keys * heads <= capacity_rows (else KVQ_ERR_CAPACITY); head_dim other
+ *                than 128 is KVQ_ERR_UNSUPPORTED.
+ *   n_keys       >= 1 cached tokens to attend to.
+ *   out          device, bf16[n_queries, heads, 128], 16-byte aligned. Written.
+ *   status       device int, set to 1 if an on-chip wait timed out (the output is then
+ *                incomplete); never cleared by the call.
+ */
+kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
+                         const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out, int* status,
+                         kvq_stream_t stream);
+
+/*
  * RTN integer codecs: the RTN_INT4 / RTN_INT2 rows of "KV Cache Quantization for
  * Self-Forcing Video Generation: A 33-Method Empirical Study", appendix Table 3
  * (symmetric blockwise quantization of K and V, block_size=16, 4-bit / 2-bit packed

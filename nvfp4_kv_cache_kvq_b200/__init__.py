@@ -66,6 +66,7 @@ def load() -> ctypes.CDLL:
         "kvq_append_batch": [CP, ctypes.POINTER(I64), ctypes.POINTER(P), I32, I64, I32, P],
         "kvq_dequantize_cache": [CP, I64, I64, P, P],
         "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
+        "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, P],
         "kvq_cache_bytes": [I32, I32, I64, I32, I64, U64P, U64P, U64P],
         "kvq_scales_to_blocked": [P, I64, I32, P, P],
         "kvq_scales_from_blocked": [P, I64, I32, P, P],
@@ -347,6 +348,28 @@ def kvq_dequantize_cache_batch(caches, row_begin: int, row_end: int, ys=None, st
     _check(load().kvq_dequantize_cache_batch(arr, ptrs, n, int(row_begin), int(row_end),
                                              _stream(stream, caches[0].device)))
     return ys
+
+
+def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: int,
+                  softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                  status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """softmax(scale * Q K^T) V per head over cache tokens [0, n_keys), K and V read from
+    their packed caches. q: bf16 [n_queries, heads, 128]; returns bf16 of q's shape.
+    ``status`` (int32, one element, device) is set to 1 if an on-chip wait timed out."""
+    if q.dim() != 3:
+        raise ValueError("q must be [n_queries, heads, head_dim]")
+    n_q, heads, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    kc, vc = k_cache.struct(), v_cache.struct()
+    _check(load().kvq_attention(_dev(q, "q"), n_q, heads, ctypes.byref(kc), ctypes.byref(vc), int(n_keys),
+                                float(softmax_scale), _dev(out, "out"), _dev(status, "status"),
+                                _stream(stream, q.device)))
+    return out
 
 
 def kvq_cache_bytes(layers: int, heads: int, capacity_tokens: int, head_dim: int, tokens_per_chunk: int):

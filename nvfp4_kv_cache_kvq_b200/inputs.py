@@ -16,6 +16,8 @@ Generation", runs a Wan2.1 stack, Table 2):
 * ``rollout`` -- per step, 30 layers x {K, V} chunks of [1560, 12, 128] (token-major),
   Student-t(4); seed step*60 + tensor.
 * ``sweep``   -- [T, 128] N(0, 1) for T = 2^10 .. 2^26; seed T.
+* ``queries`` -- attention queries of one frame [1560, 12, 128] (token-major), N(0, 1);
+  seed 1_000_000 + step (the pages give no query statistics; N(0, 1) is the plainest).
 
 Everything is drawn in fp32 with ``torch.Generator`` and rounded to bf16 by torch.
 Student-t(nu) for integer nu is drawn as Z / sqrt(chi2_nu / nu), with chi2_nu the sum
@@ -87,6 +89,11 @@ def rollout_chunk(step: int, tensor: int, heads: int = 12, tokens: int = TOKENS_
                   device="cpu") -> torch.Tensor:
     """bf16 [tokens, heads, 128] (token-major), Student-t(4), seed step*60 + tensor."""
     return student_t((tokens, heads, HEAD_DIM), 4, step * 60 + tensor, device)
+
+
+def queries(step: int, heads: int = 12, tokens: int = TOKENS_PER_FRAME, device="cpu") -> torch.Tensor:
+    """bf16 [tokens, heads, 128] (token-major), N(0, 1), seed 1_000_000 + step."""
+    return normal((tokens, heads, HEAD_DIM), 1_000_000 + step, device)
 
 
 def sweep(tokens: int, device="cpu") -> torch.Tensor:

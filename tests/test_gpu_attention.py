@@ -1,0 +1,148 @@
+"""Parity of the fused consumer kvq_attention (softmax attention reading K and V from
+their NVFP4 caches) against the fp64 oracle attention over the oracle's own dequantized
+cache.
+
+Tolerance, derived from the kernel's arithmetic: Q K^T is exact products summed in fp32;
+P = exp2(s - m) is rounded to bf16 (relative error <= 2^-9 per element) before P V, whose
+sums are fp32; the output O / l is rounded to bf16 (<= 2^-9 relative). The P rounding moves
+the output by at most 2^-9 * sum_i p_i |v_i| / l, i.e. 2^-9 times the attention of |V|,
+which the oracle computes. The bound used, 2^-8 * (attn(|V|) + |out|) + 2^-20, doubles both
+terms to absorb the fp32 accumulation and exp2 errors (below 1e-4 relative at these
+magnitudes). With a single key the result is exact: p = 1, so out is that key's V row,
+value for value as the oracle dequantizes it."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_kv_cache_kvq_b200 as kvq
+from gpu_helpers import assert_same
+from nvfp4_kv_cache_kvq_b200 import inputs
+from nvfp4_kv_cache_kvq_b200.inputs import bits
+
+pytestmark = pytest.mark.gpu
+D = 128
+
+
+def _filled_caches(orc, heads, n_tokens, tokens_per_chunk, rule, seed):
+    """A K and a V cache of n_tokens tokens appended chunk by chunk on the GPU and in the
+    oracle from the same inputs; returns (gpu caches, oracle caches)."""
+    rpc = tokens_per_chunk * heads
+    n_chunks = -(-n_tokens // tokens_per_chunk)
+    caches = [kvq.KVCache(n_chunks * rpc, rpc, D) for _ in range(2)]
+    ocs = [orc.Cache(n_chunks * rpc, rpc, D) for _ in range(2)]
+    for c in range(n_chunks):
+        toks = min(tokens_per_chunk, n_tokens - c * tokens_per_chunk)
+        for t in range(2):
+            x = inputs.student_t((toks, heads, D), 4, seed + 2 * c + t, "cuda")
+            kvq.kvq_append(caches[t], c * rpc, x, rule)
+            assert ocs[t].append(c * rpc, bits(x), rule) == 0
+    torch.cuda.synchronize()
+    for t in range(2):
+        assert_same(caches[t].packed.cpu().numpy(), ocs[t].packed, "packed cache")
+        assert_same(caches[t].scales.cpu().numpy(), ocs[t].scales, "cache scales")
+    return caches, ocs
+
+
+def _abs_bits(b: np.ndarray) -> np.ndarray:
+    return (b & 0x7FFF).astype(np.uint16)
+
+
+def _check_close(orc, got: torch.Tensor, qb, kb, vb, n_q, n_keys, heads, scale):
+    want = orc.attention(qb, kb, vb, n_q, n_keys, heads, D, scale)
+    mag = orc.attention(qb, kb, _abs_bits(vb), n_q, n_keys, heads, D, scale)
+    g = got.float().cpu().numpy().astype(np.float64).reshape(want.shape)
+    tol = 2.0 ** -8 * (mag + np.abs(want)) + 2.0 ** -20
+    err = np.abs(g - want)
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, (f"{len(bad)} of {err.size} outside tolerance; first {bad[:4].tolist()}: "
+                           f"got {g[tuple(bad[0])]} want {want[tuple(bad[0])]} tol {tol[tuple(bad[0])]}")
+    assert np.isfinite(g).all()
+
+
+@pytest.mark.parametrize("n_q,heads,tokens_per_chunk", [(1, 1, 1), (130, 3, 7), (256, 2, 64)])
+def test_single_key_returns_v_row_exactly(orc, n_q, heads, tokens_per_chunk):
+    caches, ocs = _filled_caches(orc, heads, 2 * tokens_per_chunk, tokens_per_chunk, "mse", 11)
+    q = inputs.normal((n_q, heads, D), 5, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], 1, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    v0 = ocs[1].dequantize(0, heads).reshape(heads, D)  # token 0, every head
+    want = np.broadcast_to(v0, (n_q, heads, D)).reshape(-1)
+    # equal values; a -0 of V may come out +0 (the MMA adds the masked keys' +0 products)
+    got = bits(out)
+    got_f = (got.astype(np.uint32) << 16).view(np.float32)
+    want_f = (want.astype(np.uint32) << 16).view(np.float32)
+    bad = np.nonzero(got_f != want_f)[0]
+    assert bad.size == 0, (f"{bad.size} of {got.size} differ; first at {bad[:8].tolist()}: "
+                           f"got {got[bad[:8]].tolist()} want {want[bad[:8]].tolist()}")
+
+
+@pytest.mark.parametrize("n_q,heads,n_keys,tokens_per_chunk,rule", [
+    (1, 1, 1, 1, "static_6"),
+    (130, 3, 200, 50, "mse"),       # ragged query and key tiles, chunks inside a tile
+    (128, 2, 384, 128, "static_6"),  # exact tiles
+    (257, 2, 129, 64, "static_4"),   # one key past a tile
+    (64, 4, 1000, 100, "mse"),
+])
+def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rule):
+    caches, ocs = _filled_caches(orc, heads, n_keys, tokens_per_chunk, rule, 100)
+    q = inputs.normal((n_q, heads, D), 7, "cuda")
+    scale = D ** -0.5
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
+    _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, scale)
+
+
+def test_attention_peaked_scores(orc):
+    """Large scores: the running max moves between key tiles, so O is rescaled."""
+    heads, n_keys, n_q = 2, 640, 128
+    caches, ocs = _filled_caches(orc, heads, n_keys, 128, "mse", 300)
+    q = (inputs.normal((n_q, heads, D), 9, "cuda").float() * 4).to(torch.bfloat16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, 1.0, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
+    _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, 1.0)
+
+
+def test_attention_rollout_shape_sampled(orc):
+    """The rollout's attention at full size -- one frame of 1560 queries x 12 heads over a
+    60-frame cache (93,600 keys) appended frame by frame with the mse rule -- checked on a
+    sample of query rows (the oracle computes those rows only)."""
+    heads, tpc, frames = 12, inputs.TOKENS_PER_FRAME, 60
+    rpc = tpc * heads
+    caches = [kvq.KVCache(frames * rpc, rpc, D) for _ in range(2)]
+    ocs = [orc.Cache(frames * rpc, rpc, D) for _ in range(2)]
+    for step in range(frames):
+        for t in range(2):
+            x = inputs.rollout_chunk(step, t, heads, device="cuda")
+            kvq.kvq_append(caches[t], step * rpc, x, "mse")
+            assert ocs[t].append(step * rpc, bits(x), "mse") == 0
+    q = inputs.queries(frames - 1, heads, device="cuda")
+    n_keys = frames * tpc
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = torch.tensor([0, 1, 127, 128, 777, 1400, 1535, 1559])
+    kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
+    _check_close(orc, out[rows.cuda()], bits(q[rows.cuda()]), kb, vb, len(rows), n_keys, heads, D ** -0.5)
+
+
+def test_attention_argument_errors():
+    c = kvq.KVCache(64, 16, D)
+    q = torch.zeros((4, 2, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(kvq.KvqError):  # rows_per_chunk 16 is not a multiple of 3 heads
+        kvq.kvq_attention(torch.zeros((4, 3, D), dtype=torch.bfloat16, device="cuda"), c, c, 4)
+    with pytest.raises(kvq.KvqError):  # 33 keys x 2 heads > 64 rows
+        kvq.kvq_attention(q, c, c, 33)
+    with pytest.raises(kvq.KvqError):  # no keys
+        kvq.kvq_attention(q, c, c, 0)
+    c64 = kvq.KVCache(64, 16, 64)
+    with pytest.raises(kvq.KvqError):  # head_dim 64 unsupported
+        kvq.kvq_attention(torch.zeros((4, 2, 64), dtype=torch.bfloat16, device="cuda"), c64, c64, 4)

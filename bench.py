@@ -494,6 +494,8 @@ class Attention:
         self.layers, self.heads, self.tokens, self.frames, self.D = 30, 12, 1560, 60, 128
         if args.small:
             self.layers, self.heads, self.tokens, self.frames = 2, 2, 120, 6
+        if args.layers:
+            self.layers = args.layers
         self.rule = args.rule or "mse"
         self.rank = rank
         self.rpc = self.tokens * self.heads
@@ -519,6 +521,8 @@ class Attention:
         self.q = torch.stack([inputs.queries(l + self.layers * self.rank, heads=self.heads, tokens=self.tokens,
                                              device=dev) for l in range(self.layers)])
         self.o = torch.empty_like(self.q)
+        self.ws = torch.empty(kvq.kvq_attention_workspace_bytes(self.tokens, self.heads, self.n_keys),
+                              dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.kvq = kvq
         torch.cuda.synchronize()
@@ -529,8 +533,9 @@ class Attention:
         def attn():
             for l in range(self.layers):
                 kvq.kvq_attention(self.q[l], self.caches[2 * l], self.caches[2 * l + 1], self.n_keys,
-                                  out=self.o[l], status=self.status)
-        seg = Segment("attention", attn, self.layers, self.layers * self.bytes_layer, h2d=(self.q,))
+                                  out=self.o[l], workspace=self.ws, status=self.status)
+        launches = self.layers * (2 if self.ws.numel() else 1)  # attention (+ combine) per layer
+        seg = Segment("attention", attn, launches, self.layers * self.bytes_layer, h2d=(self.q,))
         seg.flops = self.layers * self.flops_layer
         return [seg]
 
@@ -748,6 +753,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=1 << 24, help="rows of the sweep workload")
     ap.add_argument("--bits", type=int, choices=(2, 4), default=4, help="bits of the rtn workload")
     ap.add_argument("--small", action="store_true", help="a reduced shape of the workload (for tests)")
+    ap.add_argument("--layers", type=int, default=None, help="layers of the attention workload (profiling)")
     ap.add_argument("--no-graphs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -815,7 +821,7 @@ def main():
         tpeak, tsrc = tensor_peak()
         roofline = {"bound": "tensor", "kernel": dom, "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
                     "frac": tflops / tpeak, "peak_source": tsrc, "traffic": None,
-                    "flops_per_launch": dom_flops / kind_launch[dom], "launches_per_step": kind_launch[dom],
+                    "flops_per_step": dom_flops, "launches_per_step": kind_launch[dom],
                     "ms_per_step": dom_ms, "hbm_GB_s": achieved}
     else:
         per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,

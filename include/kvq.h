@@ -219,16 +219,25 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
  *   q            device, bf16[n_queries, heads, 128] (token-major), 16-byte aligned.
  *   k_cache,     host pointers to the K and V cache views: rows are token * heads + head,
  *   v_cache      head_dim 128, rows_per_chunk a multiple of heads and equal in both,
- *                n_keys * heads <= capacity_rows (else KVQ_ERR_CAPACITY); head_dim other
- *                than 128 is KVQ_ERR_UNSUPPORTED.
+ *                n_keys * heads <= capacity_rows (else KVQ_ERR_CAPACITY); packed 16-byte,
+ *                scales 8-byte aligned; head_dim other than 128 is KVQ_ERR_UNSUPPORTED.
  *   n_keys       >= 1 cached tokens to attend to.
+ *   softmax_scale  positive and finite (e.g. 1/sqrt(128)).
  *   out          device, bf16[n_queries, heads, 128], 16-byte aligned. Written.
+ *   workspace    device scratch for the partial results of key splits, 16-byte aligned,
+ *                workspace_bytes long; may be NULL with 0 bytes. The call splits the keys
+ *                over more work units (to fill the GPU) only as far as the workspace
+ *                holds their partials; kvq_attention_workspace_bytes gives the size that
+ *                allows the split it would choose on the current device.
  *   status       device int, set to 1 if an on-chip wait timed out (the output is then
  *                incomplete); never cleared by the call.
+ * kvq_attention_workspace_bytes -- host only: that size for these sizes (0 when no split
+ *   would be used).
  */
 kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
-                         const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out, int* status,
-                         kvq_stream_t stream);
+                         const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out, void* workspace,
+                         uint64_t workspace_bytes, int* status, kvq_stream_t stream);
+kvq_status kvq_attention_workspace_bytes(int32_t n_queries, int32_t heads, int64_t n_keys, uint64_t* bytes);
 
 /*
  * RTN integer codecs: the RTN_INT4 / RTN_INT2 rows of "KV Cache Quantization for

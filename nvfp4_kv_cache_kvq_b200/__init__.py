@@ -66,7 +66,8 @@ def load() -> ctypes.CDLL:
         "kvq_append_batch": [CP, ctypes.POINTER(I64), ctypes.POINTER(P), I32, I64, I32, P],
         "kvq_dequantize_cache": [CP, I64, I64, P, P],
         "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
-        "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, P],
+        "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, ctypes.c_uint64, P, P],
+        "kvq_attention_workspace_bytes": [I32, I32, I64, U64P],
         "kvq_cache_bytes": [I32, I32, I64, I32, I64, U64P, U64P, U64P],
         "kvq_scales_to_blocked": [P, I64, I32, P, P],
         "kvq_scales_from_blocked": [P, I64, I32, P, P],
@@ -350,11 +351,21 @@ def kvq_dequantize_cache_batch(caches, row_begin: int, row_end: int, ys=None, st
     return ys
 
 
+def kvq_attention_workspace_bytes(n_queries: int, heads: int, n_keys: int) -> int:
+    """Workspace bytes that let kvq_attention split the keys as it would on this device."""
+    b = ctypes.c_uint64()
+    _check(load().kvq_attention_workspace_bytes(int(n_queries), int(heads), int(n_keys), ctypes.byref(b)))
+    return b.value
+
+
 def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: int,
                   softmax_scale: float | None = None, out: torch.Tensor | None = None,
-                  status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                  workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
     """softmax(scale * Q K^T) V per head over cache tokens [0, n_keys), K and V read from
     their packed caches. q: bf16 [n_queries, heads, 128]; returns bf16 of q's shape.
+    ``workspace`` (uint8, device) holds key-split partials; None allocates the size
+    kvq_attention_workspace_bytes recommends, an empty tensor forbids splitting.
     ``status`` (int32, one element, device) is set to 1 if an on-chip wait timed out."""
     if q.dim() != 3:
         raise ValueError("q must be [n_queries, heads, head_dim]")
@@ -363,12 +374,16 @@ def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: i
         softmax_scale = d ** -0.5
     if out is None:
         out = torch.empty_like(q)
+    if workspace is None:
+        workspace = torch.empty(kvq_attention_workspace_bytes(n_q, heads, n_keys), dtype=torch.uint8,
+                                device=q.device)
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace.numel() else None
     kc, vc = k_cache.struct(), v_cache.struct()
     _check(load().kvq_attention(_dev(q, "q"), n_q, heads, ctypes.byref(kc), ctypes.byref(vc), int(n_keys),
-                                float(softmax_scale), _dev(out, "out"), _dev(status, "status"),
-                                _stream(stream, q.device)))
+                                float(softmax_scale), _dev(out, "out"), ws_ptr, workspace.numel(),
+                                _dev(status, "status"), _stream(stream, q.device)))
     return out
 
 

@@ -59,7 +59,7 @@ def _check_close(orc, got: torch.Tensor, qb, kb, vb, n_q, n_keys, heads, scale):
     assert np.isfinite(g).all()
 
 
-@pytest.mark.parametrize("n_q,heads,tokens_per_chunk", [(1, 1, 1), (130, 3, 7), (256, 2, 64)])
+@pytest.mark.parametrize("n_q,heads,tokens_per_chunk", [(1, 1, 1), (130, 3, 7), (256, 2, 64), (300, 2, 5)])
 def test_single_key_returns_v_row_exactly(orc, n_q, heads, tokens_per_chunk):
     caches, ocs = _filled_caches(orc, heads, 2 * tokens_per_chunk, tokens_per_chunk, "mse", 11)
     q = inputs.normal((n_q, heads, D), 5, "cuda")
@@ -78,19 +78,26 @@ def test_single_key_returns_v_row_exactly(orc, n_q, heads, tokens_per_chunk):
                            f"got {got[bad[:8]].tolist()} want {want[bad[:8]].tolist()}")
 
 
+def _workspace(split):
+    # "auto": the recommended workspace (keys split to fill the GPU); "none": no split
+    return None if split == "auto" else torch.empty(0, dtype=torch.uint8, device="cuda")
+
+
+@pytest.mark.parametrize("split", ["auto", "none"])
 @pytest.mark.parametrize("n_q,heads,n_keys,tokens_per_chunk,rule", [
     (1, 1, 1, 1, "static_6"),
     (130, 3, 200, 50, "mse"),       # ragged query and key tiles, chunks inside a tile
     (128, 2, 384, 128, "static_6"),  # exact tiles
-    (257, 2, 129, 64, "static_4"),   # one key past a tile
+    (257, 2, 129, 64, "static_4"),   # one key past a tile; a second query pair
     (64, 4, 1000, 100, "mse"),
+    (600, 1, 2000, 300, "mse"),      # three query pairs, the last with one partial tile
 ])
-def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rule):
+def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rule, split):
     caches, ocs = _filled_caches(orc, heads, n_keys, tokens_per_chunk, rule, 100)
     q = inputs.normal((n_q, heads, D), 7, "cuda")
     scale = D ** -0.5
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, scale, status=status)
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, scale, workspace=_workspace(split), status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
@@ -108,6 +115,14 @@ def test_attention_peaked_scores(orc):
     assert int(status.item()) == 0
     kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
     _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, 1.0)
+
+
+def test_workspace_size_and_split_agree():
+    """The recommended workspace is 0 exactly when no split is used, and a split result
+    agrees with the unsplit one (both are checked against the oracle above)."""
+    assert kvq.kvq_attention_workspace_bytes(1, 1, 1) == 0
+    b = kvq.kvq_attention_workspace_bytes(1560, 12, 93600)
+    assert b > 0 and b % (1560 * 12 * (128 * 4 + 8)) == 0
 
 
 def test_attention_rollout_shape_sampled(orc):

@@ -14,19 +14,21 @@
 // workspace and combine_kernel merges them; the split count is chosen so the units fill
 // the SMs in whole waves.
 //
-// Roles inside the CTA (416 threads):
-//   warps 0-3, 4-7  softmax of query tile 0 / 1: thread t owns row t (TMEM lane t);
-//   warps 8-11      producers: load the packed K and V of a key tile (one tile ahead, in
-//                   registers) and dequantize it into 128B-swizzled shared memory, K as
-//                   key rows and V transposed (dim rows), both K-major MMA operands;
-//   warp 12         allocates TMEM; its lane 0 issues every tcgen05.mma and commit.
+// Roles inside the CTA (512 threads, 4 warps per SM sub-partition):
+//   warps 0-3, 4-7  softmax of query tile 0 / 1: thread t owns row t (TMEM lane t). Lane 0
+//                   of each warpgroup also issues that tile's tcgen05.mma and commits:
+//                   P V(j) and S(j+1) follow its own softmax, which waits on them anyway.
+//                   Warp 0 allocates and frees the TMEM.
+//   warps 8-15      producers: load the packed K and V of a key tile (the next one while
+//                   the current is consumed, in registers) and dequantize it into
+//                   128B-swizzled shared memory as key rows: K is the K-major B operand of
+//                   Q K^T, V the MN-major B operand of P V.
 // TMEM (512 columns, fp32): S0, S1 at columns 0 and 128; O0, O1 at 256 and 384.
-// The MMA thread issues, per key tile j: PV0(j), S0(j+1), PV1(j), S1(j+1), so each query
-// tile's softmax overlaps the other tile's MMAs (the ping-pong of FlashAttention-4 on
-// Blackwell). The softmax keeps a reference row max and rescales O only when the max
-// grows by more than 2^8 (exact in real arithmetic: O and l share the reference). Every
-// wait is bounded (1 s); on a timeout the kernel records an error, lets its MMAs drain,
-// frees its TMEM and returns.
+// Each query tile's softmax overlaps the other tile's MMAs (the ping-pong of
+// FlashAttention-4 on Blackwell). The softmax keeps a reference row max and rescales O
+// only when the max grows by more than 2^8 (exact in real arithmetic: O and l share the
+// reference). Every wait is bounded (1 s); on a timeout the kernel records an error, lets
+// its MMAs drain, frees its TMEM and returns.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -43,14 +45,13 @@ constexpr int kQT = 2;    // query tiles per CTA
 constexpr int kBN = 128;  // keys per tile
 constexpr int kD = 128;   // head_dim (the only one supported)
 constexpr int kSoftmaxThreads = kQT * 128;
-constexpr int kProducerThreads = 128;
-constexpr int kMmaWarp = (kSoftmaxThreads + kProducerThreads) / 32;  // 12
-constexpr int kAttnThreads = (kMmaWarp + 1) * 32;                   // 416
-// (13 warps: the SM sub-partition that holds 4 of them caps registers at 128 per thread)
+constexpr int kProducerThreads = 256;
+constexpr int kAttnThreads = kSoftmaxThreads + kProducerThreads;  // 512: 4 warps per SM sub-partition
+constexpr int kPieces = 4 * kBN / kProducerThreads;                 // 16-byte pieces per producer thread
 constexpr int kTileBytes = 32768;  // one 128 x 128 bf16 operand
-// dynamic shared memory: Q0, Q1, K, V^T, P0, P1 (each 1024-aligned)
-constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = 3 * kTileBytes, kOffP = 4 * kTileBytes;
-constexpr int kSmemBytes = 6 * kTileBytes + 1024;  // + alignment slack
+// dynamic shared memory: Q0, Q1, K stages 0 and 1, V, P0, P1 (each 1024-aligned)
+constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = 4 * kTileBytes, kOffP = 5 * kTileBytes;
+constexpr int kSmemBytes = 7 * kTileBytes + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 1000000000ull;  // give up on an mbarrier after 1 s
 constexpr float kRescaleLog2 = 8.0f;          // rescale O when the row max grows by > 2^8
@@ -60,9 +61,9 @@ constexpr uint64_t kPartialBytesPerRow = kD * 4 + 8;
 
 // mbarriers
 enum {
-    kKFull, kKEmpty, kVFull, kVEmpty,
-    kSFull0, kSFull1, kPFull0, kPFull1, kODone0, kODone1,
-    kDone, kNumBars
+    kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull, kVEmpty,
+    kSFull0, kSFull1, kPFull0, kPFull1, kODone0, kODone1, kDone0, kDone1,
+    kNumBars
 };
 
 struct AttnArgs {
@@ -102,27 +103,50 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
            (2ull << 61);
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate, bf16 A and B, both
-// K-major, M = 128, N = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
+// Descriptor of a 128B-swizzled MN-major operand: rows of 64 contiguous MN elements, one
+// row per K index; 8-row (K) groups 1024 B apart (stride byte offset) and the second
+// 64-element MN half 16 KB away (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr)
+{
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (1024ull << 16) | (64ull << 32) | (1ull << 46) |
+           (2ull << 61);
+}
 
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate, bf16 A and B, A
+// K-major, M = 128, N = 128; B K-major (kIdesc) or MN-major (kIdescBmn, bit 16).
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
+constexpr uint32_t kIdescBmn = kIdesc | (1u << 16);
+
+template <uint32_t IDESC>
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, bool accumulate)
 {
     asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 ::"r"(tmem_d), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate ? 1u : 0u)
+                 ::"r"(tmem_d), "l"(a), "l"(b), "r"(IDESC), "r"(accumulate ? 1u : 0u)
                  : "memory");
 }
 
-// D (TMEM) (+)= A[128 x 128] B[128 x 128]^T, both K-major in shared memory, as 8 MMAs of K = 16.
-__device__ __forceinline__ void mma_tile(uint32_t tmem_d, uint32_t a_base, uint32_t b_base, bool accumulate)
+// S (TMEM) = Q[128 x 128] K[128 x 128]^T, both K-major in shared memory, as 8 MMAs of K = 16.
+__device__ __forceinline__ void mma_qk(uint32_t tmem_d, uint32_t q_base, uint32_t k_base)
 {
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            mma_bf16(tmem_d, sw128_desc(a_base + kb * 16384 + s * 32), sw128_desc(b_base + kb * 16384 + s * 32),
-                     accumulate || kb > 0 || s > 0);
+            mma_bf16<kIdesc>(tmem_d, sw128_desc(q_base + kb * 16384 + s * 32),
+                             sw128_desc(k_base + kb * 16384 + s * 32), kb > 0 || s > 0);
+}
+
+// O (TMEM) (+)= P[128 x 128 keys] V[128 keys x 128]: P K-major, V row-major (key rows, the
+// MN-major B operand); key step t of 16 keys starts 2048 B (two 8-row groups) further.
+__device__ __forceinline__ void mma_pv(uint32_t tmem_d, uint32_t p_base, uint32_t v_base, bool accumulate)
+{
+#pragma unroll
+    for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16<kIdescBmn>(tmem_d, sw128_desc(p_base + kb * 16384 + s * 32),
+                                sw128_mn_desc(v_base + (kb * 4 + s) * 2048), accumulate || kb > 0 || s > 0);
 }
 
 __device__ __forceinline__ void commit(uint32_t mbar)
@@ -194,6 +218,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32])
         v[i] = __uint_as_float(r[i]);
 }
 
+// 16 columns of this warp's 32 TMEM lanes, without the wait: the registers are valid
+// only after tmem_wait_ld() and must not be read before it.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t addr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_st32(uint32_t addr, const float (&v)[32])
 {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
@@ -218,11 +256,6 @@ __device__ __forceinline__ float ex2(float x)
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {
     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-__device__ __forceinline__ void st_shared_v2(uint32_t addr, uint32_t a, uint32_t b)
-{
-    asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
 // ------------------------------------------------------------------ dequantization
@@ -252,105 +285,231 @@ __device__ __forceinline__ float block_scale(uint32_t codes, int byte, float gs)
 
 // The packed bytes of one key tile a producer thread dequantizes: one key's whole K row
 // (8 blocks), and 4 consecutive keys x 2 blocks (32 dims) of V.
-struct RawTile {
-    uint4 kc[4];      // K codes, 64 bytes
-    uint2 ksc;        // K scale codes, blocks 0..7
-    float kgs;        // K global scale of the key
-    uint4 vc[4];      // V codes of keys 0..3 (2 blocks = 16 bytes each)
-    uint32_t vsc[2];  // V scale codes: key k's two bytes at bits 16*(k&1) of vsc[k>>1]
-    float vgs[4];
+// Loads of the next tile, issued where they stand: volatile, so the compiler cannot sink
+// them past the waits that follow (they are the prefetch).
+__device__ __forceinline__ uint4 prefetch_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t prefetch_u16(const void* p)
+{
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float prefetch_f32(const float* p)
+{
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// A producer thread's share of one tensor's key tile: kPieces pieces, piece i = 16 bytes
+// (2 blocks) of the row of key (p / 4) + 64 i, quarter q = p % 4 of the row (dims 32 q ..
+// 32 q + 31). A warp's loads thus cover 8 whole 64-byte rows each. Nothing is computed
+// from the loaded values here (they are the prefetch of the next tile and must not stall
+// the thread): keys past n_kv load row 0 instead and are zeroed at dequantization by
+// `valid`, and gs = amax / 2688 is taken there too.
+struct RawPieces {
+    uint4 c[kPieces];       // codes
+    uint32_t sc[kPieces];   // scale-code pair (blocks 2q, 2q+1) in the low 16 bits
+    float amax[kPieces];    // chunk amax of the key
 };
 
-__device__ __forceinline__ float global_scale(const float* amax, int64_t key, int64_t tokens_per_chunk)
+__device__ __forceinline__ float global_scale(float amax) { return __fdiv_rn(amax, 2688.0f); }
+
+// Keys and chunk indices fit in 32 bits (a cache holds at most 2^36 elements, i.e. 2^29
+// rows of 128).
+__device__ __forceinline__ void load_pieces(const uint8_t* packed, const uint8_t* scales, const float* amax,
+                                            const AttnArgs& a, int h, int64_t key0, int p, RawPieces& r)
 {
-    return __fdiv_rn(__ldg(amax + key / tokens_per_chunk), 2688.0f);
+    const int q = p & 3;
+#pragma unroll
+    for (int i = 0; i < kPieces; ++i) {
+        int64_t key = key0 + (p >> 2) + (kBN / kPieces) * i;
+        key = key < a.n_kv ? key : 0;
+        const int64_t off = (key * a.heads + h) * 64 + 16 * q;
+        const uint32_t chunk = static_cast<uint32_t>(key) / static_cast<uint32_t>(a.tokens_per_chunk);
+        r.c[i] = prefetch_v4(packed + off);
+        r.sc[i] = prefetch_u16(scales + off / 8);
+        r.amax[i] = prefetch_f32(amax + chunk);
+    }
 }
 
-// Producer p's share of key tile [key0, key0 + 128): K row of key key0 + p; V keys
-// key0 + 4*(p%32) .. +3, dims 32*(p/32) .. +31. Keys past n_kv read as zero codes.
-__device__ __forceinline__ void load_tile(const AttnArgs& a, int h, int64_t key0, int p, RawTile& r)
+// Bit i set when piece i's key is below n_kv.
+__device__ __forceinline__ uint32_t valid_pieces(const AttnArgs& a, int64_t key0, int p)
 {
-    const int64_t H = a.heads;
-    const int64_t kkey = key0 + p;
-    if (kkey < a.n_kv) {
-        const int64_t row = kkey * H + h;
-        const uint8_t* src = a.kp + row * 64;
+    uint32_t m = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            r.kc[i] = ld_nc_v4(src + 16 * i);
-        r.ksc = ld_nc_v2(a.ks + row * 8);
-        r.kgs = global_scale(a.ka, kkey, a.tokens_per_chunk);
-    } else {
+    for (int i = 0; i < kPieces; ++i)
+        m |= (key0 + (p >> 2) + (kBN / kPieces) * i < a.n_kv ? 1u : 0u) << i;
+    return m;
+}
+
+// The four pieces dequantized into their rows of a 128B-swizzled tile (K as the K-major
+// B operand of Q K^T, V as the MN-major B operand of P V: the same bytes); invalid keys
+// get gs = 0, i.e. zeros. Threads of quarters 2 and 3 store their two blocks in swapped
+// order, so the 8 threads of each shared-memory wavefront hit 8 different 16-byte bank
+// groups.
+__device__ __forceinline__ void store_pieces(const RawPieces& r, uint32_t valid, int p, uint32_t sT)
+{
+    const int q = p & 3, kb = q >> 1, swap = q & 2;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            r.kc[i] = make_uint4(0u, 0u, 0u, 0u);
-        r.ksc = make_uint2(0u, 0u);
-        r.kgs = 0.0f;
+    for (int i = 0; i < kPieces; ++i) {
+        const int row = (p >> 2) + (kBN / kPieces) * i;
+        const float gs = (valid >> i) & 1u ? global_scale(r.amax[i]) : 0.0f;
+        const float SA = block_scale(r.sc[i], swap ? 1 : 0, gs), SB = block_scale(r.sc[i], swap ? 0 : 1, gs);
+        const uint4 c = r.c[i];
+        uint32_t y0[4], y1[4], y2[4], y3[4];
+        dequant8(swap ? c.z : c.x, SA, y0);
+        dequant8(swap ? c.w : c.y, SA, y1);
+        dequant8(swap ? c.x : c.z, SB, y2);
+        dequant8(swap ? c.y : c.w, SB, y3);
+        const int ch = (q & 1) * 4;
+        st_shared_v4(sT + sw128(row, kb, ch + (0 ^ swap)), y0[0], y0[1], y0[2], y0[3]);
+        st_shared_v4(sT + sw128(row, kb, ch + (1 ^ swap)), y1[0], y1[1], y1[2], y1[3]);
+        st_shared_v4(sT + sw128(row, kb, ch + (2 ^ swap)), y2[0], y2[1], y2[2], y2[3]);
+        st_shared_v4(sT + sw128(row, kb, ch + (3 ^ swap)), y3[0], y3[1], y3[2], y3[3]);
     }
-    const int quad = p & 31, quarter = p >> 5;
-    r.vsc[0] = r.vsc[1] = 0u;
+}
+
+// ------------------------------------------------------------------ softmax pieces
+
+// Max of row S over the tile's valid keys (MASK: only the first `valid`), in four
+// independent chains.
+template <bool MASK>
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int valid)
+{
+    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        float s[32];
+        tmem_ld32(tS + c * 32, s);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int64_t key = key0 + 4 * quad + k;
-        if (key < a.n_kv) {
-            const int64_t row = key * H + h;
-            r.vc[k] = ld_nc_v4(a.vp + row * 64 + quarter * 16);
-            const uint32_t sc = __ldg(reinterpret_cast<const uint16_t*>(a.vs + row * 8 + quarter * 2));
-            r.vsc[k >> 1] |= sc << (16 * (k & 1));
-            r.vgs[k] = global_scale(a.va, key, a.tokens_per_chunk);
+        for (int i = 0; i < 32; ++i)
+            if (!MASK || c * 32 + i < valid)
+                m[i & 3] = fmaxf(m[i & 3], s[i]);
+    }
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), written
+// as bf16 to row r of P (K-major, 128B-swizzled); returns the fp32 sum of p.
+// 2^x for a pair of fp32 on the FMA pipe (so that the ex2 unit, which the other half of
+// the elements use, is not the bottleneck): Cody and Waite's range reduction x = n + f,
+// n = round(x), |f| <= 1/2, then 2^f by a degree-3 polynomial fitted to the relative
+// error on [-1/2, 1/2] (max relative error 7.5e-5, far below P's bf16 rounding of 2^-9),
+// and 2^n added to the exponent field. x is clamped below at -125 (2^-125 next to the row
+// maximum's 1 is nothing); callers keep x below 2^22.
+__device__ __forceinline__ uint64_t exp2_poly(uint64_t x2)
+{
+    float x0, x1;
+    f32x2_unpack(x2, x0, x1);
+    x2 = f32x2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t one2 = f32x2_pack(1.0f, 1.0f), mone2 = f32x2_pack(-1.0f, -1.0f);
+    const uint64_t magic2 = f32x2_pack(12582912.0f, 12582912.0f), nmagic2 = f32x2_pack(-12582912.0f, -12582912.0f);
+    const uint64_t t = f32x2_fma(x2, one2, magic2);  // 1.5 * 2^23 + round(x): round(x) in the low bits
+    const uint64_t f = f32x2_fma(f32x2_fma(t, one2, nmagic2), mone2, x2);  // x - round(x)
+    uint64_t p = f32x2_fma(f32x2_pack(0.0551716685f, 0.0551716685f), f, f32x2_pack(0.2426111400f, 0.2426111400f));
+    p = f32x2_fma(p, f, f32x2_pack(0.6932609677f, 0.6932609677f));
+    p = f32x2_fma(p, f, f32x2_pack(0.9999280572f, 0.9999280572f));
+    float t0, t1, p0, p1;
+    f32x2_unpack(t, t0, t1);
+    f32x2_unpack(p, p0, p1);
+    p0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    p1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+    return f32x2_pack(p0, p1);
+}
+
+// 16 columns (chunk c) of the row: p into P, sums into the packed accumulators; with
+// TRACK also the max of the raw scores into mt. Columns 0-7 of the chunk take the ex2
+// unit, columns 8-15 the polynomial.
+template <bool MASK, bool TRACK>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[16], int c, uint32_t sP, int r, int valid,
+                                          uint64_t sc2, uint64_t nm2, uint64_t& la, uint64_t& lb, float& mt)
+{
+    const uint64_t one2 = f32x2_pack(1.0f, 1.0f);
+    uint32_t pw[8];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+        const float s0 = __uint_as_float(sr[i]), s1 = __uint_as_float(sr[i + 1]);
+        if (TRACK) {
+            if (!MASK || c * 16 + i < valid)
+                mt = fmaxf(mt, s0);
+            if (!MASK || c * 16 + i + 1 < valid)
+                mt = fmaxf(mt, s1);
+        }
+        const uint64_t x2 = f32x2_fma(f32x2_pack(s0, s1), sc2, nm2);
+        float p0, p1;
+        if (i < 8) {
+            float x0, x1;
+            f32x2_unpack(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
         } else {
-            r.vc[k] = make_uint4(0u, 0u, 0u, 0u);
-            r.vgs[k] = 0.0f;
+            f32x2_unpack(exp2_poly(x2), p0, p1);
         }
+        if (MASK) {
+            if (c * 16 + i >= valid)
+                p0 = 0.0f;
+            if (c * 16 + i + 1 >= valid)
+                p1 = 0.0f;
+        }
+        if ((i >> 1) & 1)
+            lb = f32x2_fma(f32x2_pack(p0, p1), one2, lb);
+        else
+            la = f32x2_fma(f32x2_pack(p0, p1), one2, la);
+        pw[i >> 1] = bf16x2_from_f32(p1, p0);
     }
+    const int kb = c >> 2, ch0 = (c & 3) * 2;
+    st_shared_v4(sP + sw128(r, kb, ch0), pw[0], pw[1], pw[2], pw[3]);
+    st_shared_v4(sP + sw128(r, kb, ch0 + 1), pw[4], pw[5], pw[6], pw[7]);
 }
 
-// K row p of the tile into sK (key rows, dims contiguous, K-major).
-__device__ __forceinline__ void store_k(const RawTile& r, int p, uint32_t sK)
+// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), written
+// as bf16 to row r of P (K-major, 128B-swizzled); returns the fp32 sum of p and, with
+// TRACK, the max of the raw scores in mt. The TMEM load of the next 16 columns is in
+// flight while the current ones are computed.
+template <bool MASK, bool TRACK>
+__device__ __forceinline__ float tile_row_exp(uint32_t tS, uint32_t sP, int r, int valid, float scale_log2, float m,
+                                              float& mt)
 {
-#pragma unroll
-    for (int b = 0; b < 8; ++b) {
-        const float S = block_scale(b < 4 ? r.ksc.x : r.ksc.y, b & 3, r.kgs);
-        const uint4 c = r.kc[b >> 1];
-        uint32_t y0[4], y1[4];
-        dequant8((b & 1) ? c.z : c.x, S, y0);
-        dequant8((b & 1) ? c.w : c.y, S, y1);
-        const int kb = b >> 2, ch = 2 * (b & 3);
-        st_shared_v4(sK + sw128(p, kb, ch), y0[0], y0[1], y0[2], y0[3]);
-        st_shared_v4(sK + sw128(p, kb, ch + 1), y1[0], y1[1], y1[2], y1[3]);
+    const uint64_t sc2 = f32x2_pack(scale_log2, scale_log2), nm2 = f32x2_pack(-m, -m);
+    uint64_t la = 0, lb = 0;  // two packed partial sums (+0.0 bit patterns)
+    uint32_t r0[16], r1[16];
+    mt = -INFINITY;
+    tmem_ld16_async(tS, r0);
+    tmem_wait_ld();
+#pragma unroll 1
+    for (int k = 0; k < 4; ++k) {
+        const int c = 2 * k;
+        tmem_ld16_async(tS + (c + 1) * 16, r1);
+        exp_chunk<MASK, TRACK>(r0, c, sP, r, valid, sc2, nm2, la, lb, mt);
+        tmem_wait_ld();
+        if (k < 3)
+            tmem_ld16_async(tS + (c + 2) * 16, r0);
+        exp_chunk<MASK, TRACK>(r1, c + 1, sP, r, valid, sc2, nm2, la, lb, mt);
+        if (k < 3)
+            tmem_wait_ld();
     }
+    float a0, a1, b0, b1;
+    f32x2_unpack(la, a0, a1);
+    f32x2_unpack(lb, b0, b1);
+    return __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(b0, b1));
 }
 
-// V of 4 keys x 32 dims into sVt (dim rows, keys contiguous, K-major): per dim, the four
-// keys' values as one 8-byte store.
-__device__ __forceinline__ void store_v(const RawTile& r, int p, uint32_t sV)
+template <bool TRACK>
+__device__ __forceinline__ float row_exp(uint32_t tS, uint32_t sP, int r, int valid, float scale_log2, float m,
+                                         float& mt)
 {
-    const int quad = p & 31, quarter = p >> 5;
-    const int kb = quad >> 4, chunk = (quad & 15) >> 1, byte = (quad & 1) * 8;
-#pragma unroll
-    for (int bb = 0; bb < 2; ++bb) {
-        uint32_t y[4][8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float S = block_scale(r.vsc[k >> 1] >> (16 * (k & 1)), bb, r.vgs[k]);
-            uint32_t lo[4], hi[4];
-            dequant8(bb ? r.vc[k].z : r.vc[k].x, S, lo);
-            dequant8(bb ? r.vc[k].w : r.vc[k].y, S, hi);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                y[k][i] = lo[i];
-                y[k][4 + i] = hi[i];
-            }
-        }
-#pragma unroll
-        for (int dp = 0; dp < 8; ++dp) {
-            const int d = quarter * 32 + bb * 16 + 2 * dp;
-            st_shared_v2(sV + sw128(d, kb, chunk) + byte, __byte_perm(y[0][dp], y[1][dp], 0x5410),
-                         __byte_perm(y[2][dp], y[3][dp], 0x5410));
-            st_shared_v2(sV + sw128(d + 1, kb, chunk) + byte, __byte_perm(y[0][dp], y[1][dp], 0x7632),
-                         __byte_perm(y[2][dp], y[3][dp], 0x7632));
-        }
-    }
+    return valid == kBN ? tile_row_exp<false, TRACK>(tS, sP, r, valid, scale_log2, m, mt)
+                        : tile_row_exp<true, TRACK>(tS, sP, r, valid, scale_log2, m, mt);
 }
 
 // ------------------------------------------------------------------ kernels
@@ -374,8 +533,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
     const uint32_t base = (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) + 1023u) & ~1023u;
     const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(&bars[0]));
     auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+    const uint32_t sV = base + kOffV;
+    // key tile j lives in K stage j % 2; its barriers' phase is j / 2
+    auto sK = [base](int j) { return base + kOffK + static_cast<uint32_t>(j & 1) * kTileBytes; };
+    auto kfull = [&bar](int j) { return bar(kKFull0 + (j & 1)); };
+    auto kempty = [&bar](int j) { return bar(kKEmpty0 + (j & 1)); };
 
-    if (warp == kMmaWarp) {
+    if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          static_cast<uint32_t>(__cvta_generic_to_shared(&tmem_base_s))),
                      "r"(kTmemCols)
@@ -383,17 +547,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(bar(kKFull), kProducerThreads);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(bar(kKFull0 + st), kProducerThreads);
+            mbar_init(bar(kKEmpty0 + st), n_qt);  // one commit per active query tile's issuer
+        }
         mbar_init(bar(kVFull), kProducerThreads);
-        mbar_init(bar(kKEmpty), 1);
-        mbar_init(bar(kVEmpty), 1);
-        mbar_init(bar(kSFull0), 1);
-        mbar_init(bar(kSFull1), 1);
-        mbar_init(bar(kPFull0), 128);
-        mbar_init(bar(kPFull1), 128);
-        mbar_init(bar(kODone0), 1);
-        mbar_init(bar(kODone1), 1);
-        mbar_init(bar(kDone), 1);
+        mbar_init(bar(kVEmpty), n_qt);
+        for (int g = 0; g < kQT; ++g) {
+            mbar_init(bar(kSFull0 + g), 1);
+            mbar_init(bar(kPFull0 + g), 128);
+            mbar_init(bar(kODone0 + g), 1);
+            mbar_init(bar(kDone0 + g), 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // both query tiles -> shared memory (rows past n_q are zero)
@@ -412,38 +577,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
     const uint32_t tmem = tmem_base_s;
 
     if (tid < kSoftmaxThreads) {
-        // ---------------------------------------------------------------- softmax
+        // ---------------------------------------------------------------- softmax + MMA issue
+        // Lane 0 of the warpgroup's first warp issues this query tile's MMAs: S_g(j+1) and
+        // P_g V(j) follow its own softmax, which waits on them anyway.
         const int g = tid >> 7, r = tid & 127;
         if (g < n_qt) {
             const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
             const uint32_t tS = tmem + g * 128 + lane_off, tO = tmem + 256 + g * 128 + lane_off;
-            const uint32_t sP = base + kOffP + g * kTileBytes;
+            const uint32_t sQ = base + kOffQ + g * kTileBytes, sP = base + kOffP + g * kTileBytes;
             const uint32_t bS = bar(kSFull0 + g), bP = bar(kPFull0 + g), bO = bar(kODone0 + g);
+            const bool issuer = r == 0;
             float m_run = -INFINITY, l_run = 0.0f;
             bool ok = true;
-            for (int j = 0; j < n_tiles; ++j) {
+            if (issuer && n_tiles > 0) {
+                ok = wait_phase(kfull(0), 0);
+                if (ok) {
+                    tc_after_sync();
+                    mma_qk(tmem + g * 128, sQ, sK(0));
+                    commit(bS);
+                    commit(kempty(0));
+                }
+            }
+            for (int j = 0; ok && j < n_tiles; ++j) {
                 ok = warp_wait(bS, j & 1);
                 if (!ok)
                     break;
                 tc_after_sync();
                 const int64_t key0 = static_cast<int64_t>(t_begin + j) * kBN;
                 const int valid = static_cast<int>(a.n_kv - key0 < kBN ? a.n_kv - key0 : kBN);
-                // pass 1: the row max of this tile
-                float mt = -INFINITY;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float s[32];
-                    tmem_ld32(tS + c * 32, s);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c * 32 + i < valid)
-                            mt = fmaxf(mt, s[i]);
-                }
-                mt = __fmul_rn(mt, a.scale_log2);
-                const float m_cand = fmaxf(m_run, mt);
-                const bool need = m_cand > m_run + kRescaleLog2;
-                const float m_use = need ? m_cand : m_run;
-                const float alpha = need ? ex2(m_run - m_use) : 1.0f;
                 // P and O of this query tile are free once the previous P V is done
                 if (j > 0) {
                     ok = warp_wait(bO, (j - 1) & 1);
@@ -451,27 +612,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                         break;
                     tc_after_sync();
                 }
-                // pass 2: P = bf16(2^(s * scale_log2 - m)) into row r of P (K-major)
-                float lt = 0.0f;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float s[32];
-                    tmem_ld32(tS + c * 32, s);
-                    uint32_t pw[16];
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float p0 = c * 32 + i < valid ? ex2(__fmaf_rn(s[i], a.scale_log2, -m_use)) : 0.0f;
-                        const float p1 =
-                            c * 32 + i + 1 < valid ? ex2(__fmaf_rn(s[i + 1], a.scale_log2, -m_use)) : 0.0f;
-                        lt = __fadd_rn(lt, p0);
-                        lt = __fadd_rn(lt, p1);
-                        pw[i >> 1] = bf16x2_from_f32(p1, p0);
+                float m_use, alpha, lt, mt;
+                bool need;
+                if (j == 0) {
+                    // no reference yet: the row max first, then P
+                    m_use = __fmul_rn(valid == kBN ? tile_row_max<false>(tS, valid) : tile_row_max<true>(tS, valid),
+                                      a.scale_log2);
+                    alpha = 0.0f;
+                    need = true;
+                    lt = row_exp<false>(tS, sP, r, valid, a.scale_log2, m_use, mt);
+                } else {
+                    // P against the reference max, tracking this tile's max; only when
+                    // that max exceeds the reference by more than 2^8 (rare once the
+                    // first tiles are seen) is P recomputed against it and O rescaled
+                    lt = row_exp<true>(tS, sP, r, valid, a.scale_log2, m_run, mt);
+                    const float m_cand = fmaxf(m_run, __fmul_rn(mt, a.scale_log2));
+                    need = m_cand > m_run + kRescaleLog2;
+                    m_use = need ? m_cand : m_run;
+                    alpha = need ? ex2(m_run - m_use) : 1.0f;
+                    if (__any_sync(0xFFFFFFFFu, need)) {
+                        const float lt2 = row_exp<false>(tS, sP, r, valid, a.scale_log2, m_use, mt);
+                        lt = need ? lt2 : lt;
                     }
-                    const int kb = c >> 1, ch0 = (c & 1) * 4;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        st_shared_v4(sP + sw128(r, kb, ch0 + u), pw[4 * u], pw[4 * u + 1], pw[4 * u + 2],
-                                     pw[4 * u + 3]);
                 }
                 l_run = __fmaf_rn(l_run, alpha, lt);
                 m_run = m_use;
@@ -490,6 +652,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                 fence_async_smem();
                 tc_before_sync();
                 mbar_arrive(bP);
+                if (issuer) {
+                    // O_g += P_g V(j), then S_g(j+1) = Q_g K(j+1)^T
+                    ok = wait_phase(bP, j & 1) && wait_phase(bar(kVFull), j & 1);
+                    if (ok) {
+                        tc_after_sync();
+                        mma_pv(tmem + 256 + g * 128, sP, sV, j > 0);
+                        commit(bO);
+                        commit(bar(kVEmpty));
+                        if (j + 1 < n_tiles) {
+                            ok = wait_phase(kfull(j + 1), ((j + 1) >> 1) & 1);
+                            if (ok) {
+                                tc_after_sync();
+                                mma_qk(tmem + g * 128, sQ, sK(j + 1));
+                                commit(bS);
+                                commit(kempty(j + 1));
+                            }
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             }
             if (ok && n_tiles > 0) {
                 ok = warp_wait(bO, (n_tiles - 1) & 1);
@@ -526,82 +708,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                         a.part_ml[prow] = make_float2(m_run, l_run);
                 }
             }
+            if (issuer) {
+                commit(bar(kDone0 + g));  // completes once every MMA this thread issued has
+                if (!wait_phase(bar(kDone0 + g), 0))
+                    ok = false;
+            }
             if (!ok && lane == 0)
                 atomicExch(a.status, 1);
         }
-    } else if (warp < kMmaWarp) {
+    } else {
         // ---------------------------------------------------------------- producers
+        // K runs one key tile ahead of V (K has two stages): K(j+1) is stored before V(j),
+        // so Q K^T of the next tile never waits for the V buffer, which P V(j-1) holds.
+        // Each tensor's raw pieces are refilled right after its tile is stored, so the
+        // loads land while the other tensor is dequantized and the barriers are awaited.
         const int p = tid - kSoftmaxThreads;
-        const uint32_t sK = base + kOffK, sV = base + kOffV;
-        RawTile cur, nxt;
-        bool ok = true;
-        if (n_tiles > 0)
-            load_tile(a, h, static_cast<int64_t>(t_begin) * kBN, p, cur);
-        for (int j = 0; j < n_tiles; ++j) {
-            if (j + 1 < n_tiles)
-                load_tile(a, h, static_cast<int64_t>(t_begin + j + 1) * kBN, p, nxt);
-            if (j > 0 && !(ok = wait_phase(bar(kKEmpty), (j - 1) & 1)))
-                break;
-            store_k(cur, p, sK);
-            fence_async_smem();
-            mbar_arrive(bar(kKFull));
-            if (j > 0 && !(ok = wait_phase(bar(kVEmpty), (j - 1) & 1)))
-                break;
-            store_v(cur, p, sV);
-            fence_async_smem();
-            mbar_arrive(bar(kVFull));
-            cur = nxt;
-        }
-        if (!ok && lane == 0)
-            atomicExch(a.status, 1);
-    } else if (lane == 0) {
-        // ---------------------------------------------------------------- MMA issue
+        auto key0_of = [&](int j) { return static_cast<int64_t>(t_begin + j) * kBN; };
+        RawPieces rk, rv;
         bool ok = true;
         if (n_tiles > 0) {
-            ok = wait_phase(bar(kKFull), 0);
-            if (ok) {
-                tc_after_sync();
-                for (int g = 0; g < n_qt; ++g) {
-                    mma_tile(tmem + g * 128, base + kOffQ + g * kTileBytes, base + kOffK, false);
-                    commit(bar(kSFull0 + g));
-                }
-                commit(bar(kKEmpty));
-            }
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                if (!(ok = wait_phase(bar(kVFull), j & 1)))
-                    break;
-                tc_after_sync();
-                for (int g = 0; g < n_qt; ++g) {
-                    if (!(ok = wait_phase(bar(kPFull0 + g), j & 1)))
-                        break;
-                    tc_after_sync();
-                    mma_tile(tmem + 256 + g * 128, base + kOffP + g * kTileBytes, base + kOffV, j > 0);
-                    commit(bar(kODone0 + g));
-                    if (g == n_qt - 1)
-                        commit(bar(kVEmpty));
-                    if (j + 1 < n_tiles) {
-                        if (g == 0) {
-                            if (!(ok = wait_phase(bar(kKFull), (j + 1) & 1)))
-                                break;
-                            tc_after_sync();
-                        }
-                        mma_tile(tmem + g * 128, base + kOffQ + g * kTileBytes, base + kOffK, false);
-                        commit(bar(kSFull0 + g));
-                        if (g == n_qt - 1)
-                            commit(bar(kKEmpty));
-                    }
-                }
-            }
+            load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(0), p, rk);
+            load_pieces(a.vp, a.vs, a.va, a, h, key0_of(0), p, rv);
+            store_pieces(rk, valid_pieces(a, key0_of(0), p), p, sK(0));
+            fence_async_smem();
+            mbar_arrive(kfull(0));
+            if (n_tiles > 1)
+                load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(1), p, rk);
         }
-        commit(bar(kDone));  // completes once every MMA issued above has
-        if (!wait_phase(bar(kDone), 0))
-            ok = false;
-        if (!ok)
+        for (int j = 0; j < n_tiles; ++j) {
+            if (j + 1 < n_tiles) {
+                // stage (j+1) % 2 was last read by the S MMAs of key tile j - 1
+                if (j > 0 && !(ok = wait_phase(kempty(j + 1), (((j + 1) >> 1) - 1) & 1)))
+                    break;
+                store_pieces(rk, valid_pieces(a, key0_of(j + 1), p), p, sK(j + 1));
+                fence_async_smem();
+                mbar_arrive(kfull(j + 1));
+                if (j + 2 < n_tiles)
+                    load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(j + 2), p, rk);
+            }
+            if (j > 0 && !(ok = wait_phase(bar(kVEmpty), (j - 1) & 1)))
+                break;
+            store_pieces(rv, valid_pieces(a, key0_of(j), p), p, sV);
+            fence_async_smem();
+            mbar_arrive(bar(kVFull));
+            if (j + 1 < n_tiles)
+                load_pieces(a.vp, a.vs, a.va, a, h, key0_of(j + 1), p, rv);
+        }
+        if (!ok && lane == 0)
             atomicExch(a.status, 1);
     }
     tc_before_sync();
     __syncthreads();
-    if (warp == kMmaWarp)
+    if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
 }
 

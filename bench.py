@@ -482,6 +482,92 @@ class Rtn(Sweep):
         return nbytes, time.perf_counter() - t0, f"first {m} of {self.tokens} rows, {reps} repetitions"
 
 
+class Recent:
+    """The rollout under the RECENT2 cache policy of the Self-Forcing study (RTN_INT4
+    RECENT2): every frame appends 1560 tokens per layer to 30 layers x {K, V} through
+    kvq_recent_append_batch (the frame leaving the two-frame bf16 window is RTN
+    INT4-quantized into the prefix) and reads every layer's whole cache back through
+    kvq_recent_read_batch (prefix dequantized, bf16 tail copied)."""
+    name = "recent"
+
+    def __init__(self, args, rank):
+        self.layers, self.heads, self.tokens, self.frames, self.D, self.R, self.bits = 30, 12, 1560, 60, 128, 2, 4
+        if args.small:
+            self.layers, self.heads, self.tokens, self.frames = 2, 2, 120, 6
+        self.rank = rank
+        self.rpc = self.tokens * self.heads
+        self.chunk_elems = self.rpc * self.D
+        self.config = {
+            "workload": f"rollout with the RECENT2 policy (RTN INT4 prefix, newest {self.R} frames bf16): "
+                        f"{self.layers} layers x {{K,V}}, {self.heads} heads, {self.tokens} tokens/frame x "
+                        f"{self.frames} frames, head_dim {self.D}, Student-t(4)",
+            "model": "Wan-shaped self-forcing KV cache (synthetic)", "global_batch": 1,
+            "seq_len": self.tokens * self.frames, "parallelism": "replica per GPU",
+            "l2": "inputs larger than L2 (per-step appends and the growing cache exceed 126 MB)",
+        }
+
+    def setup(self, kvq, inputs, dev):
+        T = 2 * self.layers
+        self.caches = [kvq.RecentCache(self.frames, self.rpc, self.D, self.bits, self.R, dev) for _ in range(T)]
+        self.x = torch.empty((self.frames, T, self.chunk_elems), dtype=torch.bfloat16, device=dev)
+        for f in range(self.frames):
+            for t in range(T):
+                self.x[f, t] = inputs.rollout_chunk(f + self.frames * self.rank, t, heads=self.heads,
+                                                    tokens=self.tokens, device=dev).reshape(-1)
+        cap = self.frames * self.chunk_elems
+        self.yk = torch.empty(cap, dtype=torch.bfloat16, device=dev)
+        self.yv = torch.empty(cap, dtype=torch.bfloat16, device=dev)
+        self.kvq = kvq
+
+    def segments(self):
+        kvq, T, segs = self.kvq, 2 * self.layers, []
+        bq = 2.0 + self.bits / 8 + 2.0 / 16  # RTN quantize: bf16 read, codes + bf16 scale written
+        for f in range(self.frames):
+            xs = [self.x[f, t] for t in range(T)]
+            evict = f >= self.R
+
+            def app(f=f, xs=xs):
+                kvq.kvq_recent_append_batch(self.caches, f, xs)
+            # RTN quantize of the evicted frame (once the window is full) + the bf16 copy
+            segs.append(Segment("recent_append", app, math.ceil(T / kvq.MAX_BATCH) * (2 if evict else 1),
+                                T * self.chunk_elems * ((bq if evict else 0.0) + 4.0), h2d=(self.x[f],)))
+            n = f + 1
+            r = min(self.R, n)
+            prefix = n - r
+
+            def rd(n=n):
+                for l in range(self.layers):
+                    kvq.kvq_recent_read_batch(self.caches[2 * l:2 * l + 2], n,
+                                              [self.yk[:n * self.chunk_elems], self.yv[:n * self.chunk_elems]])
+            segs.append(Segment("recent_read", rd, self.layers * ((1 if prefix else 0) + 1),
+                                T * self.chunk_elems * (prefix * bq + r * 4.0)))
+        return segs
+
+    def d2h(self):
+        return [self.caches[0].packed, self.caches[0].scales, self.caches[0].recent]
+
+    def tokens_per_step(self):
+        return self.tokens * self.frames
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        """Layer 0's K and V through the rollout until the time budget is spent."""
+        caches = [orc.RecentCache(self.rpc, self.D, self.bits, self.R) for _ in range(2)]
+        bq = 2.0 + self.bits / 8 + 2.0 / 16
+        spent, nbytes, f = 0.0, 0.0, 0
+        while f < self.frames and spent < budget_s:
+            for t in range(2):
+                xb = inputs.bits(inputs.rollout_chunk(f, t, heads=self.heads, tokens=self.tokens))
+                t1 = time.perf_counter()
+                caches[t].append(xb)
+                caches[t].read()
+                spent += time.perf_counter() - t1
+                n = f + 1
+                r = min(self.R, n)
+                nbytes += self.chunk_elems * ((bq if f >= self.R else 0.0) + 4.0 + (n - r) * bq + r * 4.0)
+            f += 1
+        return nbytes, spent, f"layer 0 K and V (2 of {2 * self.layers} tensors), frames 1..{f} of the rollout"
+
+
 class Attention:
     """The rollout's attention at its last frame, reading the packed cache directly: for
     every layer, one frame of 1560 queries x 12 heads attends to that layer's 60-frame
@@ -599,7 +685,7 @@ class Attention:
         return self.bytes_layer * m / self.tokens, dt, f"layer 0, {m} of {self.tokens} query rows"
 
 
-WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention)}
+WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention, Recent)}
 
 
 # ---------------------------------------------------------------------------- runner
@@ -826,9 +912,9 @@ def main():
     else:
         per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
                     "roundtrip": B_AMAX + B_QUANT + 2.0, "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16,
-                    "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}[dom]
-        tb = measured_traffic(dom)
-        elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom]
+                    "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}.get(dom)
+        tb = measured_traffic(dom) if per_elem else None
+        elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom] if per_elem else None
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",
                     "traffic": None if tb is None else tb * elems_per_launch,

@@ -273,6 +273,56 @@ kvq_status kvq_rtn_dequantize_batch(const uint8_t* const* packed, const uint16_t
                                     kvq_stream_t stream);
 
 /*
+ * RECENT cache policy: the RTN_INT4 RECENT2 method of "KV Cache Quantization for
+ * Self-Forcing Video Generation" (appendix Table 3): the newest `recent_blocks` (2)
+ * frame-blocks of a K or V cache are kept in bf16 ("recent_k / recent_v" state) and only
+ * older blocks are RTN-quantized; a read dequantizes the quantized prefix and copies the
+ * bf16 tail back in. A frame-block is rows_per_block rows (tokens x heads) of head_dim.
+ *   packed   device, RTN codes of capacity_blocks blocks: capacity_blocks * rows_per_block
+ *            * head_dim * bits / 8 bytes (block b at offset b * its size), 2*bits-aligned.
+ *   scales   device, bf16 scales, one per 16 elements, same block order, 2-byte aligned.
+ *   recent   device, bf16 ring of recent_blocks blocks (block b in slot b % recent_blocks),
+ *            32-byte aligned.
+ * head_dim is a positive multiple of 16 with rows_per_block * head_dim a multiple of 16;
+ * bits is 4 (the study's RECENT2 prefix) or 2.
+ */
+typedef struct {
+    uint8_t* packed;
+    uint16_t* scales;
+    void* recent;
+    int64_t capacity_blocks;
+    int64_t rows_per_block;
+    int32_t head_dim;
+    int32_t bits;
+    int32_t recent_blocks;
+} kvq_recent_cache;
+
+/*
+ * kvq_recent_append_batch -- quantize-on-write of frame-block `block` into n_caches
+ *   caches (e.g. every layer's K and V), blocks appended in order 0, 1, 2, ...: the
+ *   block leaving the bf16 window (block - recent_blocks, if block >= recent_blocks) is
+ *   RTN-quantized from its ring slot into the prefix, then x takes that slot.
+ *   caches  host array of n_caches cache views (same rows_per_block, head_dim, bits,
+ *           recent_blocks).
+ *   xs      host array of n_caches device pointers, bf16[rows_per_block * head_dim] each,
+ *           32-byte aligned.
+ *   block < capacity_blocks, else KVQ_ERR_CAPACITY.
+ */
+kvq_status kvq_recent_append_batch(const kvq_recent_cache* caches, int32_t n_caches, int64_t block,
+                                   const void* const* xs, kvq_stream_t stream);
+
+/*
+ * kvq_recent_read_batch -- the whole active cache of n_caches caches as bf16, n_blocks
+ *   being the number of blocks appended so far (not checked; at most capacity_blocks,
+ *   else KVQ_ERR_CAPACITY): blocks [0, n_blocks - r) dequantized from the prefix,
+ *   r = min(recent_blocks, n_blocks), then the r newest blocks copied from the ring.
+ *   ys  host array of n_caches device pointers, bf16[n_blocks * rows_per_block *
+ *       head_dim] each, 32-byte aligned. Written.
+ */
+kvq_status kvq_recent_read_batch(const kvq_recent_cache* caches, int32_t n_caches, int64_t n_blocks,
+                                 void* const* ys, kvq_stream_t stream);
+
+/*
  * Blocked scale layout: the 128 x 4 tiles block-scaled MMA operands read ("How NVFP4
  * Quantization Works in LongLive 2.0", "Stage 3", step 1: the dequantizer first undoes
  * it, "from_blocked"). A [rows, cols] matrix of one-byte scales (row-major: the scales

@@ -31,6 +31,12 @@ class KvqError(RuntimeError):
         self.status = status
 
 
+class _RecentCache(ctypes.Structure):
+    _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("recent", ctypes.c_void_p),
+                ("capacity_blocks", ctypes.c_int64), ("rows_per_block", ctypes.c_int64), ("head_dim", ctypes.c_int32),
+                ("bits", ctypes.c_int32), ("recent_blocks", ctypes.c_int32)]
+
+
 class _Cache(ctypes.Structure):
     _fields_ = [("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("amax", ctypes.c_void_p),
                 ("capacity_rows", ctypes.c_int64), ("rows_per_chunk", ctypes.c_int64),
@@ -68,6 +74,8 @@ def load() -> ctypes.CDLL:
         "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
         "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, ctypes.c_uint64, P, P],
         "kvq_attention_workspace_bytes": [I32, I32, I64, U64P],
+        "kvq_recent_append_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
+        "kvq_recent_read_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
         "kvq_cache_bytes": [I32, I32, I64, I32, I64, U64P, U64P, U64P],
         "kvq_scales_to_blocked": [P, I64, I32, P, P],
         "kvq_scales_from_blocked": [P, I64, I32, P, P],
@@ -385,6 +393,52 @@ def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: i
                                 float(softmax_scale), _dev(out, "out"), ws_ptr, workspace.numel(),
                                 _dev(status, "status"), _stream(stream, q.device)))
     return out
+
+
+class RecentCache:
+    """A K or V cache under the RECENT policy (RTN_INT4 RECENT2 of the Self-Forcing study):
+    the newest ``recent_blocks`` frame-blocks in a bf16 ring, older blocks RTN-quantized
+    (``bits``) in the prefix. A frame-block is ``rows_per_block`` rows of ``head_dim``."""
+
+    def __init__(self, capacity_blocks: int, rows_per_block: int, head_dim: int = 128, bits: int = 4,
+                 recent_blocks: int = 2, device="cuda"):
+        self.capacity_blocks, self.rows_per_block, self.head_dim = int(capacity_blocks), int(rows_per_block), int(head_dim)
+        self.bits, self.recent_blocks = int(bits), int(recent_blocks)
+        elems = self.rows_per_block * self.head_dim
+        self.packed = torch.zeros(self.capacity_blocks * elems * self.bits // 8, dtype=torch.uint8, device=device)
+        self.scales = torch.zeros(self.capacity_blocks * elems // BLOCK, dtype=torch.bfloat16, device=device)
+        self.recent = torch.zeros(self.recent_blocks * elems, dtype=torch.bfloat16, device=device)
+        self.device = self.packed.device
+
+    def struct(self) -> _RecentCache:
+        return _RecentCache(_dev(self.packed, "packed"), _dev(self.scales, "scales"), _dev(self.recent, "recent"),
+                            self.capacity_blocks, self.rows_per_block, self.head_dim, self.bits, self.recent_blocks)
+
+
+def kvq_recent_append_batch(caches, block: int, xs, stream=None):
+    """Quantize-on-write of frame-block ``block`` (bf16, rows_per_block x head_dim each)."""
+    n = len(caches)
+    if len(xs) != n:
+        raise ValueError("caches and xs differ in length")
+    if n == 0:
+        return
+    arr = (_RecentCache * n)(*[c.struct() for c in caches])
+    ptrs = (ctypes.c_void_p * n)(*[_dev(x, "x") for x in xs])
+    _check(load().kvq_recent_append_batch(arr, n, int(block), ptrs, _stream(stream, caches[0].device)))
+
+
+def kvq_recent_read_batch(caches, n_blocks: int, ys=None, stream=None):
+    """The first n_blocks frame-blocks of each cache as bf16 (prefix dequantized, tail copied)."""
+    n = len(caches)
+    if n == 0:
+        return []
+    if ys is None:
+        ys = [torch.empty(n_blocks * c.rows_per_block * c.head_dim, dtype=torch.bfloat16, device=c.device)
+              for c in caches]
+    arr = (_RecentCache * n)(*[c.struct() for c in caches])
+    ptrs = (ctypes.c_void_p * n)(*[_dev(y, "y") for y in ys])
+    _check(load().kvq_recent_read_batch(arr, n, int(n_blocks), ptrs, _stream(stream, caches[0].device)))
+    return ys
 
 
 def kvq_cache_bytes(layers: int, heads: int, capacity_tokens: int, head_dim: int, tokens_per_chunk: int):

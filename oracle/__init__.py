@@ -216,6 +216,31 @@ def rtn_dequantize(packed: np.ndarray, scales: np.ndarray, head_dim: int, bits: 
     return y
 
 
+# ---- RECENT cache policy ---------------------------------------------------------------
+
+class RecentCache:
+    """The RTN_INT4 RECENT2 cache policy of the Self-Forcing study (appendix Table 3),
+    step by step: the newest `recent_blocks` frame-blocks are kept as bf16 state; when a
+    block is appended, the block falling out of that window is RTN-quantized (bits) into
+    the prefix; a read dequantizes the prefix and appends the bf16 tail."""
+
+    def __init__(self, rows_per_block: int, head_dim: int, bits: int = 4, recent_blocks: int = 2):
+        self.rows_per_block, self.head_dim, self.bits, self.recent_blocks = rows_per_block, head_dim, bits, recent_blocks
+        self.prefix = []  # (packed, scales) of quantized blocks 0, 1, ...
+        self.recent = []  # bf16 bit patterns of the newest blocks, oldest first
+
+    def append(self, x_bits: np.ndarray):
+        x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1)
+        assert x_bits.size == self.rows_per_block * self.head_dim
+        self.recent.append(x_bits.copy())
+        if len(self.recent) > self.recent_blocks:
+            self.prefix.append(rtn_quantize(self.recent.pop(0), self.head_dim, self.bits))
+
+    def read(self) -> np.ndarray:
+        parts = [rtn_dequantize(p, s, self.head_dim, self.bits) for p, s in self.prefix] + list(self.recent)
+        return np.concatenate(parts) if parts else np.zeros(0, np.uint16)
+
+
 # ---- blocked scale layout ----------------------------------------------------------
 
 def blocked_bytes(rows: int, cols: int) -> int:

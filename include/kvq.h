@@ -240,6 +240,28 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
 kvq_status kvq_attention_workspace_bytes(int32_t n_queries, int32_t heads, int64_t n_keys, uint64_t* bytes);
 
 /*
+ * kvq_attention_noalloc -- kvq_attention without a workspace argument, for callers that
+ *   cannot allocate device memory: code running inside a host framework that owns the
+ *   GPU's memory through its own pool and budget (a cudaMalloc there would bypass its
+ *   accounting or fail under its limit), or a latency-critical loop that cannot afford
+ *   cudaMalloc's implicit device synchronization. It allocates nothing: the partial
+ *   results of the key split live in a 32 MiB array built into the library, which every
+ *   GPU that runs the attention kernels holds until the process exits. (The pages have
+ *   no counterpart; this is a deployment convenience of this library.)
+ *   Arguments, result and errors are those of kvq_attention, plus:
+ *   - sizes whose key split needs more than 32 MiB (kvq_attention_workspace_bytes above
+ *     32 MiB) return KVQ_ERR_CAPACITY with the needed size in kvq_last_error();
+ *   - the first call on a device looks up the array's device address (once per device,
+ *     that device current); make that first call before any stream capture;
+ *   - every call on a GPU shares the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race on it and must be ordered by the caller. Nothing
+ *     in it needs to start at zero.
+ */
+kvq_status kvq_attention_noalloc(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
+                                 const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out,
+                                 int* status, kvq_stream_t stream);
+
+/*
  * RTN integer codecs: the RTN_INT4 / RTN_INT2 rows of "KV Cache Quantization for
  * Self-Forcing Video Generation: A 33-Method Empirical Study", appendix Table 3
  * (symmetric blockwise quantization of K and V, block_size=16, 4-bit / 2-bit packed

@@ -74,6 +74,7 @@ def load() -> ctypes.CDLL:
         "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
         "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, ctypes.c_uint64, P, P],
         "kvq_attention_workspace_bytes": [I32, I32, I64, U64P],
+        "kvq_attention_noalloc": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, P],
         "kvq_recent_append_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
         "kvq_recent_read_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
         "kvq_cache_bytes": [I32, I32, I64, I32, I64, U64P, U64P, U64P],
@@ -392,6 +393,29 @@ def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: i
     _check(load().kvq_attention(_dev(q, "q"), n_q, heads, ctypes.byref(kc), ctypes.byref(vc), int(n_keys),
                                 float(softmax_scale), _dev(out, "out"), ws_ptr, workspace.numel(),
                                 _dev(status, "status"), _stream(stream, q.device)))
+    return out
+
+
+def kvq_attention_noalloc(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: int,
+                          softmax_scale: float | None = None, out: torch.Tensor | None = None,
+                          status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """kvq_attention for callers that cannot allocate device memory for a workspace: the
+    key-split partials use the library's built-in 32 MiB scratch (sizes needing more are
+    rejected). ``out`` and ``status`` are still the caller's; pass them to allocate
+    nothing here either."""
+    if q.dim() != 3:
+        raise ValueError("q must be [n_queries, heads, head_dim]")
+    n_q, heads, d = q.shape
+    if softmax_scale is None:
+        softmax_scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    kc, vc = k_cache.struct(), v_cache.struct()
+    _check(load().kvq_attention_noalloc(_dev(q, "q"), n_q, heads, ctypes.byref(kc), ctypes.byref(vc), int(n_keys),
+                                        float(softmax_scale), _dev(out, "out"), _dev(status, "status"),
+                                        _stream(stream, q.device)))
     return out
 
 

@@ -32,6 +32,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "kvq.h"
 #include "kvq_common.h"
@@ -935,6 +936,76 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
     cfg.dynamicSmemBytes = 0;
     st = launched(cudaLaunchKernelEx(&cfg, combine_kernel, a), "kvq_attention (combine)");
     return st == KVQ_OK ? ok() : st;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// kvq_attention_noalloc: kvq_attention for callers that cannot allocate device memory.
+// The key-split partials live in this file-scope array instead of a caller workspace.
+// The array is allocated with this file's kernels on every GPU that runs them and is
+// held until the process exits; every call on a GPU shares it.
+
+namespace kvq {
+namespace {
+
+constexpr uint64_t kNoAllocScratchBytes = uint64_t{32} << 20;  // 32 MiB
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) uint8_t g_attention_scratch[kNoAllocScratchBytes];
+
+// Device address of g_attention_scratch on the current device, looked up once per device
+// with that device current (in host code the array's name is only a host-side stand-in).
+kvq_status scratch_address(void** ptr)
+{
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return launched(e, "kvq_attention_noalloc (current device)");
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention_noalloc: device %d beyond the %d supported", dev, kMaxDevices);
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attention_scratch);
+        if (e != cudaSuccess)
+            return launched(e, "kvq_attention_noalloc (scratch address)");
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return KVQ_OK;
+}
+
+}  // namespace
+}  // namespace kvq
+
+extern "C" {
+
+kvq_status kvq_attention_noalloc(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
+                                 const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out,
+                                 int* status, kvq_stream_t stream)
+{
+    NvtxRange nvtx_range("kvq_attention_noalloc");
+    uint64_t need = 0;
+    kvq_status st = kvq_attention_workspace_bytes(n_queries, heads, n_keys, &need);
+    if (st != KVQ_OK)
+        return st;
+    if (need > kNoAllocScratchBytes)
+        return fail(KVQ_ERR_CAPACITY,
+                    "kvq_attention_noalloc: %d queries x %d heads over %lld keys need %llu bytes of scratch; the "
+                    "built-in scratch holds %llu (use kvq_attention with a workspace)",
+                    n_queries, heads, static_cast<long long>(n_keys), static_cast<unsigned long long>(need),
+                    static_cast<unsigned long long>(kNoAllocScratchBytes));
+    void* scratch = nullptr;
+    if (need > 0 && (st = scratch_address(&scratch)) != KVQ_OK)
+        return st;
+    // the same call as kvq_attention with the recommended workspace: the same key split,
+    // hence the same result; every partial the combine reads is written first, so the
+    // scratch needs no clearing
+    return kvq_attention(q, n_queries, heads, k_cache, v_cache, n_keys, softmax_scale, out, scratch, need, status,
+                         stream);
 }
 
 }  // extern "C"

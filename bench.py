@@ -257,10 +257,15 @@ class Layer:
     def setup(self, kvq, inputs, dev):
         self.x = [inputs.layer_kv(2 * self.rank + kv, heads=self.heads, tokens=self.tokens, device=dev)
                   for kv in (0, 1)]
-        self.p = [torch.empty(self.n // 2, dtype=torch.uint8, device=dev) for _ in range(2)]
-        self.s = [torch.empty(self.n // 16, dtype=torch.uint8, device=dev) for _ in range(2)]
-        self.a = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(2)]
-        self.y = [torch.empty(self.n, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.allocate(kvq, dev)
+
+    def allocate(self, kvq, dev):
+        """Outputs for every input tensor in self.x."""
+        m = len(self.x)
+        self.p = [torch.empty(self.n // 2, dtype=torch.uint8, device=dev) for _ in range(m)]
+        self.s = [torch.empty(self.n // 16, dtype=torch.uint8, device=dev) for _ in range(m)]
+        self.a = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(m)]
+        self.y = [torch.empty(self.n, dtype=torch.bfloat16, device=dev) for _ in range(m)]
         self.kvq = kvq
 
     def segments(self):
@@ -374,8 +379,8 @@ class Single(Layer):
         self.flush = True
 
     def setup(self, kvq, inputs, dev):
-        Layer.setup(self, kvq, inputs, dev)
         self.x = [inputs.normal((self.tokens, self.D), seed=self.rank, device=dev)]
+        self.allocate(kvq, dev)
 
     def oracle_sample(self, orc, inputs, budget_s):
         t0, nbytes, reps = time.perf_counter(), 0.0, 0
@@ -404,8 +409,8 @@ class Sweep(Layer):
                        "l2": "flushed between timed steps (256 MB write)" if self.flush else "inputs larger than L2"}
 
     def setup(self, kvq, inputs, dev):
-        Layer.setup(self, kvq, inputs, dev)
         self.x = [inputs.sweep(self.tokens, device=dev)]
+        self.allocate(kvq, dev)
 
     def oracle_sample(self, orc, inputs, budget_s):
         nbytes, reps = 0.0, 0

@@ -34,7 +34,8 @@
  * Conventions for every call:
  *   - Pointers named "device" are CUDA device (or managed) memory that the caller
  *     allocates, owns and frees. The library never allocates or frees memory and keeps
- *     no state between calls. Host pointers are read before the call returns.
+ *     no state between calls, with one stated exception: kvq_attention_noalloc's
+ *     built-in scratch array (see there). Host pointers are read before the call returns.
  *   - Work is queued on `stream` (a cudaStream_t; NULL is the legacy default stream)
  *     and runs asynchronously; results are valid once the stream has been
  *     synchronized. Calls on the same stream run in order.

@@ -402,35 +402,16 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int valid)
 
 // p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), written
 // as bf16 to row r of P (K-major, 128B-swizzled); returns the fp32 sum of p.
-// 2^x for a pair of fp32 on the FMA pipe (so that the ex2 unit, which the other half of
-// the elements use, is not the bottleneck): Cody and Waite's range reduction x = n + f,
-// n = round(x), |f| <= 1/2, then 2^f by a degree-3 polynomial fitted to the relative
-// error on [-1/2, 1/2] (max relative error 7.5e-5, far below P's bf16 rounding of 2^-9),
-// and 2^n added to the exponent field. x is clamped below at -125 (2^-125 next to the row
-// maximum's 1 is nothing); callers keep x below 2^22.
-__device__ __forceinline__ uint64_t exp2_poly(uint64_t x2)
+// max(a, b, c) in one instruction (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c)
 {
-    float x0, x1;
-    f32x2_unpack(x2, x0, x1);
-    x2 = f32x2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-    const uint64_t one2 = f32x2_pack(1.0f, 1.0f), mone2 = f32x2_pack(-1.0f, -1.0f);
-    const uint64_t magic2 = f32x2_pack(12582912.0f, 12582912.0f), nmagic2 = f32x2_pack(-12582912.0f, -12582912.0f);
-    const uint64_t t = f32x2_fma(x2, one2, magic2);  // 1.5 * 2^23 + round(x): round(x) in the low bits
-    const uint64_t f = f32x2_fma(f32x2_fma(t, one2, nmagic2), mone2, x2);  // x - round(x)
-    uint64_t p = f32x2_fma(f32x2_pack(0.0551716685f, 0.0551716685f), f, f32x2_pack(0.2426111400f, 0.2426111400f));
-    p = f32x2_fma(p, f, f32x2_pack(0.6932609677f, 0.6932609677f));
-    p = f32x2_fma(p, f, f32x2_pack(0.9999280572f, 0.9999280572f));
-    float t0, t1, p0, p1;
-    f32x2_unpack(t, t0, t1);
-    f32x2_unpack(p, p0, p1);
-    p0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    p1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-    return f32x2_pack(p0, p1);
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // 16 columns (chunk c) of the row: p into P, sums into the packed accumulators; with
-// TRACK also the max of the raw scores into mt. Columns 0-7 of the chunk take the ex2
-// unit, columns 8-15 the polynomial.
+// TRACK also the max of the raw scores into mt.
 template <bool MASK, bool TRACK>
 __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[16], int c, uint32_t sP, int r, int valid,
                                           uint64_t sc2, uint64_t nm2, uint64_t& la, uint64_t& lb, float& mt)
@@ -441,21 +422,18 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[16], int c, uint3
     for (int i = 0; i < 16; i += 2) {
         const float s0 = __uint_as_float(sr[i]), s1 = __uint_as_float(sr[i + 1]);
         if (TRACK) {
-            if (!MASK || c * 16 + i < valid)
-                mt = fmaxf(mt, s0);
-            if (!MASK || c * 16 + i + 1 < valid)
-                mt = fmaxf(mt, s1);
+            if (!MASK)
+                mt = max3(mt, s0, s1);
+            else {
+                if (c * 16 + i < valid)
+                    mt = fmaxf(mt, s0);
+                if (c * 16 + i + 1 < valid)
+                    mt = fmaxf(mt, s1);
+            }
         }
-        const uint64_t x2 = f32x2_fma(f32x2_pack(s0, s1), sc2, nm2);
-        float p0, p1;
-        if (i < 8) {
-            float x0, x1;
-            f32x2_unpack(x2, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-        } else {
-            f32x2_unpack(exp2_poly(x2), p0, p1);
-        }
+        float x0, x1;
+        f32x2_unpack(f32x2_fma(f32x2_pack(s0, s1), sc2, nm2), x0, x1);
+        float p0 = ex2(x0), p1 = ex2(x1);
         if (MASK) {
             if (c * 16 + i >= valid)
                 p0 = 0.0f;
@@ -884,6 +862,8 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
     const int64_t key_tiles = (n_keys + kBN - 1) / kBN;
     if (key_tiles > INT32_MAX)
         return fail(KVQ_ERR_INVALID_ARG, "kvq_attention: too many keys");
+    if (static_cast<int64_t>(n_queries) * heads / (kCombineThreads / 32) >= INT32_MAX)
+        return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: n_queries * heads too large");
     const int64_t qpairs = (n_queries + kQT * kBM - 1) / (kQT * kBM);
     int splits = choose_splits(qpairs * heads, static_cast<int>(key_tiles), sm_count());
     while (splits > 1 && partial_bytes(splits, n_queries, heads) > workspace_bytes)

@@ -104,6 +104,21 @@ def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rul
     _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, scale)
 
 
+def test_attention_many_key_splits(orc):
+    """One query tile of one head over 64 key tiles: the split heuristic spreads the keys
+    over the most units (up to 64), so the combine merges many partials."""
+    heads, n_keys, n_q = 1, 64 * 128 - 3, 100
+    assert kvq.kvq_attention_workspace_bytes(n_q, heads, n_keys) >= 32 * n_q * heads * (128 * 4 + 8)
+    caches, ocs = _filled_caches(orc, heads, n_keys, 1000, "mse", 500)
+    q = inputs.normal((n_q, heads, D), 11, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
+    _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, D ** -0.5)
+
+
 def test_attention_peaked_scores(orc):
     """Large scores: the running max moves between key tiles, so O is rescaled."""
     heads, n_keys, n_q = 2, 640, 128

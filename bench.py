@@ -53,15 +53,14 @@ def kernel_source_sha256() -> str:
 
     h = hashlib.sha256()
     for rel in ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_rtn.cu",
-                "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh", "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"):
+                "nvfp4_kv_cache_kvq_b200/csrc/kvq_attention.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
+                "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def measured_traffic(kind: str):
-    """DRAM bytes per element of a kernel kind from the committed ncu summary
-    (profiles/traffic.json), or None when the kernels changed since that capture."""
+def _traffic_entry(kind: str):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
@@ -69,8 +68,22 @@ def measured_traffic(kind: str):
         return None
     if t.get("source_sha256") != kernel_source_sha256():
         return None
-    k = t.get("kernels", {}).get(kind)
-    return None if k is None else float(k["dram_bytes_per_elem"])
+    return t.get("kernels", {}).get(kind)
+
+
+def measured_traffic(kind: str):
+    """DRAM bytes per element of a kernel kind from the committed ncu summary
+    (profiles/traffic.json), or None when the kernels changed since that capture."""
+    k = _traffic_entry(kind)
+    return None if k is None or "dram_bytes_per_elem" not in k else float(k["dram_bytes_per_elem"])
+
+
+def measured_launch_traffic(kind: str, shape: str):
+    """DRAM bytes of one launch of a kernel kind captured on exactly `shape`, or None."""
+    k = _traffic_entry(kind)
+    if k is None or k.get("shape") != shape:
+        return None
+    return float(k["dram_bytes_per_launch"])
 
 
 def tensor_peak():
@@ -592,6 +605,7 @@ class Attention:
         self.rpc = self.tokens * self.heads
         self.n_keys = self.tokens * self.frames
         self.flops_layer = 4.0 * self.tokens * self.n_keys * self.heads * self.D
+        self.launch_shape = f"{self.tokens} queries x {self.heads} heads x {self.n_keys} keys"
         # packed K and V (codes + scales) read once, queries read, output written
         self.bytes_layer = 2 * self.n_keys * self.heads * self.D * 0.5625 + 2 * self.rpc * self.D * 2.0
         self.config = {
@@ -911,7 +925,8 @@ def main():
         tflops = dom_flops / (dom_ms * 1e-3) / 1e12
         tpeak, tsrc = tensor_peak()
         roofline = {"bound": "tensor", "kernel": dom, "achieved": tflops, "peak": tpeak, "unit": "TFLOP/s",
-                    "frac": tflops / tpeak, "peak_source": tsrc, "traffic": None,
+                    "frac": tflops / tpeak, "peak_source": tsrc,
+                    "traffic": measured_launch_traffic(dom, getattr(wl, "launch_shape", "")),
                     "flops_per_step": dom_flops, "launches_per_step": kind_launch[dom],
                     "ms_per_step": dom_ms, "hbm_GB_s": achieved}
     else:

@@ -234,6 +234,13 @@ class Rollout:
     def tokens_per_step(self):
         return self.tokens * self.frames
 
+    def extra_rates(self, kind_ms):
+        """Appended tokens/s of the append kernels, and prefix tokens/s of the reads
+        (every layer, K and V, all heads of a token counted once)."""
+        prefix_tokens = self.tokens * self.frames * (self.frames + 1) // 2
+        return {"append_tokens_per_s": self.tokens * self.frames / (kind_ms["append"] * 1e-3),
+                "dequant_prefix_tokens_per_s": prefix_tokens / (kind_ms["dequant"] * 1e-3)}
+
     def oracle_sample(self, orc, inputs, budget_s):
         """Layer 0's K and V through the rollout until the time budget is spent."""
         caches = [orc.Cache(self.frames * self.rpc, self.rpc, self.D) for _ in range(2)]
@@ -424,6 +431,17 @@ class Sweep(Layer):
     def setup(self, kvq, inputs, dev):
         self.x = [inputs.sweep(self.tokens, device=dev)]
         self.allocate(kvq, dev)
+
+    def segments(self):
+        """quantize (amax + codes), quantize again with amax_in (codes only: the same
+        bytes, timed on their own), dequantize."""
+        segs = Layer.segments(self)
+        kvq = self.kvq
+
+        def q_in():
+            kvq.kvq_quantize_batch(self.x, self.D, self.rule, amax_in=self.a[:1], packed=self.p[:1], scales=self.s[:1])
+        segs.insert(1, Segment("quantize_amax_in", q_in, 1, self.n * B_QUANT))
+        return segs
 
     def oracle_sample(self, orc, inputs, budget_s):
         nbytes, reps = 0.0, 0
@@ -931,6 +949,7 @@ def main():
                     "ms_per_step": dom_ms, "hbm_GB_s": achieved}
     else:
         per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
+                    "quantize_amax_in": B_QUANT,
                     "roundtrip": B_AMAX + B_QUANT + 2.0, "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16,
                     "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}.get(dom)
         tb = measured_traffic(dom) if per_elem else None
@@ -951,6 +970,8 @@ def main():
             "roofline": roofline, "kernels": per_kind, "gpu_launches": sum(s.launches for s in segs) * args.steps,
             "clocks": sampler.summary(), "graphs": not args.no_graphs}
 
+    if hasattr(wl, "extra_rates"):
+        line.update(wl.extra_rates({k: kind_ms[k] / args.steps for k in kinds}))
     if hasattr(wl, "check"):
         wl.check()
     if hasattr(wl, "unfused"):

@@ -212,8 +212,8 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
  *   reading K and V straight from their NVFP4 caches: each tile of keys is dequantized
  *   in on-chip memory to the same bf16 values kvq_dequantize_cache writes, so no dense
  *   bf16 copy of the cache is ever stored ("How to Use KV Cache Quantization with
- *   LongLive's LongLiveQuantizationConfig", "CUDA De-quantization Pipeline": dequantize
- *   during the attention operation; Self-Forcing study, abstract and Figure 6: the
+ *   LongLive's LongLiveQuantizationConfig", "CUDA De-quantization Pipeline": the cache
+ *   is dequantized while attention runs; Self-Forcing study, abstract and Figure 6: the
  *   transient BF16 buffers of dequantize-then-attend set the peak memory). Every query
  *   attends to cache tokens [0, n_keys) (no mask); P is rounded to bf16 before P V and
  *   both products accumulate in fp32 on the tensor cores.

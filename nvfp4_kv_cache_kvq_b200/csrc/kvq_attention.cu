@@ -5,8 +5,8 @@
 // BF16 before attention ("KV Cache Quantization for Self-Forcing Video Generation",
 // appendix Table 3) and find that those transient BF16 buffers dominate peak memory
 // (abstract; Figure 6); "How to Use KV Cache Quantization with LongLive's
-// LongLiveQuantizationConfig" ("CUDA De-quantization Pipeline") dequantizes "during the
-// attention operation".
+// LongLiveQuantizationConfig" ("CUDA De-quantization Pipeline") dequantizes the cache while
+// attention runs.
 //
 // Work unit (one CTA): two query tiles of 128 rows of one head against one range of key
 // tiles (128 keys each). When the keys are split over several units, each leaves a

@@ -192,7 +192,8 @@ kvq_status kvq_append_batch(const kvq_cache* caches, const int64_t* row_offsets,
 /*
  * kvq_dequantize_cache -- dequantize cache rows [row_begin, row_end) to bf16, each row
  *   with the amax of its chunk ("Stage 3: KV-Cache De-quantization at Inference";
- *   appendix Table 3: dequantize the active cache back to dense BF16 before attention).
+ *   Self-Forcing study, appendix Table 3: the active cache goes back to dense BF16
+ *   before attention).
  *   y  device, bf16[(row_end - row_begin) * head_dim], 32-byte aligned. Written.
  *   row_end <= capacity_rows (else KVQ_ERR_CAPACITY).
  */

@@ -270,8 +270,8 @@ def attention(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray, n_quer
     """softmax(Q K^T * scale) V per head, in fp64, on bf16 inputs given as bit patterns:
     q [n_queries, heads, head_dim], k and v [n_keys, heads, head_dim] (token-major, the
     cache's row order). Returns fp64 [n_queries, heads, head_dim]. This is the consumer
-    the pages place after dequantization ("dequantize the active cache back to dense
-    BF16 before attention", Self-Forcing study, appendix Table 3)."""
+    the pages place after dequantization (the Self-Forcing study, appendix Table 3:
+    the active cache is turned back into dense BF16 and then attended over)."""
     def f64(b, rows):
         u = (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
         return u.astype(np.float64).reshape(rows, heads, head_dim)

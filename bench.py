@@ -49,14 +49,20 @@ L2_BYTES = 126 * 2 ** 20
 
 
 def kernel_source_sha256() -> str:
+    """SHA-256 of the measured kernels' code, comments and whitespace left out (the
+    profiles stay valid across comment edits, not across code changes)."""
     import hashlib
+    import re
 
     h = hashlib.sha256()
     for rel in ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_rtn.cu",
                 "nvfp4_kv_cache_kvq_b200/csrc/kvq_attention.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
                 "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)  # block comments
+        src = re.sub(r"//[^\n]*", " ", src)                # line comments (no source line has // in a string)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()
 
 

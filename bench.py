@@ -92,6 +92,37 @@ def measured_launch_traffic(kind: str, shape: str):
     return float(k["dram_bytes_per_launch"])
 
 
+_CUDART = None
+
+
+def memcpy2d_to_host(dst: int, dpitch: int, src: int, spitch: int, width: int, height: int, stream) -> None:
+    """cudaMemcpy2DAsync device -> pinned host on `stream` (height rows of width bytes)."""
+    global _CUDART
+    if _CUDART is None:
+        import ctypes
+        import ctypes.util
+        import glob
+
+        paths = glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
+                                       "libcudart.so*")) + [ctypes.util.find_library("cudart")]
+        for path in paths:
+            if path:
+                try:
+                    _CUDART = ctypes.CDLL(path)
+                    break
+                except OSError:
+                    pass
+        if _CUDART is None:
+            raise RuntimeError("libcudart not found")
+        f = _CUDART.cudaMemcpy2DAsync
+        f.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_size_t,
+                      ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p]
+        f.restype = ctypes.c_int
+    rc = _CUDART.cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, height, 2, stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"cudaMemcpy2DAsync failed: {rc}")
+
+
 def tensor_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -230,12 +261,37 @@ class Rollout:
             segs.append(Segment("dequant", deq, self.layers, T * rows * self.D * B_DEQUANT))
         return segs
 
-    def d2h(self):
+    def _bases(self):
         c0 = self.caches[0]
         # the three backing buffers of every cache (allocate_caches carves them contiguously)
-        return [c0.packed._base if c0.packed._base is not None else c0.packed,
-                c0.scales._base if c0.scales._base is not None else c0.scales,
-                c0.amax._base if c0.amax._base is not None else c0.amax]
+        return [t._base if t._base is not None else t for t in (c0.packed, c0.scales, c0.amax)]
+
+    def d2h(self):
+        """Copied back at the end of the step: the chunk amax of every cache (the packed
+        codes and scales go back frame by frame, see d2h_per_segment)."""
+        return [self._bases()[2]]
+
+    def d2h_per_segment(self, n_segs):
+        """After frame f's append, its packed rows and scales are final in every cache:
+        one 2D copy per buffer (a row per cache) sends them back while later frames run."""
+        packed, scales, _ = self._bases()
+        T = 2 * self.layers
+        self.packed_h = torch.empty(packed.shape, dtype=packed.dtype, pin_memory=True)
+        self.scales_h = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+        after = [None] * n_segs
+        pb, sb = self.chunk_elems // 2, self.chunk_elems // 16  # bytes of one frame in one cache
+        p_pitch, s_pitch = packed.numel() // T, scales.numel() // T
+
+        def make(f):
+            def go(stream):
+                memcpy2d_to_host(self.packed_h.data_ptr() + f * pb, p_pitch, packed.data_ptr() + f * pb, p_pitch,
+                                 pb, T, stream)
+                memcpy2d_to_host(self.scales_h.data_ptr() + f * sb, s_pitch, scales.data_ptr() + f * sb, s_pitch,
+                                 sb, T, stream)
+            return go
+        for f in range(self.frames):
+            after[2 * f] = make(f)  # segment 2f is frame f's append
+        return after, self.frames * T * (pb + sb)
 
     def tokens_per_step(self):
         return self.tokens * self.frames
@@ -856,6 +912,7 @@ def run_step(segs, events, e2e=None):
                     dst.copy_(src, non_blocking=True)
                 ready[i] = torch.cuda.Event()
                 ready[i].record(cs)
+    per_seg = e2e.get("d2h_after") if e2e is not None else None
     for i, seg in enumerate(segs):
         if i > 0:
             events[i].record()
@@ -865,9 +922,19 @@ def run_step(segs, events, e2e=None):
             seg.graph.replay()
         else:
             seg.fn()
+        if per_seg is not None and per_seg[i] is not None:
+            # this segment's final outputs go back on their own stream while the next
+            # segments compute
+            done = torch.cuda.Event()
+            done.record(main)
+            e2e["d2h_stream"].wait_event(done)
+            per_seg[i](e2e["d2h_stream"])
     if e2e is not None:
-        for dst, src in zip(e2e["d2h_dst"], e2e["d2h_src"]):
-            dst.copy_(src, non_blocking=True)
+        with torch.cuda.stream(e2e["d2h_stream"]):
+            e2e["d2h_stream"].wait_stream(main)
+            for dst, src in zip(e2e["d2h_dst"], e2e["d2h_src"]):
+                dst.copy_(src, non_blocking=True)
+        main.wait_stream(e2e["d2h_stream"])
     events[-1].record()
 
 
@@ -1015,7 +1082,13 @@ def run_e2e(args, wl, segs, bytes_step, world):
     d2h_src = wl.d2h()
     d2h_dst = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d2h_src]
     d2h_bytes = sum(t.numel() * t.element_size() for t in d2h_src)
-    e2e = {"h2d": h2d, "d2h_src": d2h_src, "d2h_dst": d2h_dst, "stream": torch.cuda.Stream()}
+    e2e = {"h2d": h2d, "d2h_src": d2h_src, "d2h_dst": d2h_dst, "stream": torch.cuda.Stream(),
+           "d2h_stream": torch.cuda.Stream()}
+    if hasattr(wl, "d2h_per_segment"):
+        # outputs that are final after a segment are copied back right after it
+        after, more_bytes = wl.d2h_per_segment(len(segs))
+        e2e["d2h_after"] = after
+        d2h_bytes += more_bytes
     events = [torch.cuda.Event(enable_timing=True) for _ in range(len(segs) + 1)]
     run_step(segs, events, e2e)
     torch.cuda.synchronize()

@@ -23,7 +23,11 @@
 //                   the current is consumed, in registers) and dequantize it into
 //                   128B-swizzled shared memory as key rows: K is the K-major B operand of
 //                   Q K^T, V the MN-major B operand of P V.
-// TMEM (512 columns, fp32): S0, S1 at columns 0 and 128; O0, O1 at 256 and 384.
+// TMEM (512 columns, fp32): S0, S1 at columns 0 and 128; O0, O1 at 256 and 384. P_g, the
+// bf16 probabilities, is written over the first 64 columns of S_g (two keys per column)
+// and is the A operand of P V straight from TMEM, so P never passes through shared
+// memory and P V reads only V there. S_g(j+1) overwrites P_g(j) only after P V(j) has
+// read it: a thread's tcgen05.mma operations run in the order it issues them.
 // Each query tile's softmax overlaps the other tile's MMAs (the ping-pong of
 // FlashAttention-4 on Blackwell). The softmax keeps a reference row max and rescales O
 // only when the max grows by more than 2^8 (exact in real arithmetic: O and l share the
@@ -50,10 +54,18 @@ constexpr int kProducerThreads = 256;
 constexpr int kAttnThreads = kSoftmaxThreads + kProducerThreads;  // 512: 4 warps per SM sub-partition
 constexpr int kPieces = 4 * kBN / kProducerThreads;                 // 16-byte pieces per producer thread
 constexpr int kTileBytes = 32768;  // one 128 x 128 bf16 operand
-// dynamic shared memory: Q0, Q1, K stages 0 and 1, V, P0, P1 (each 1024-aligned)
-constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = 4 * kTileBytes, kOffP = 5 * kTileBytes;
-constexpr int kSmemBytes = 7 * kTileBytes + 1024;  // + alignment slack
+// dynamic shared memory: Q0, Q1, K stages 0 and 1, V (each 1024-aligned)
+constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = 4 * kTileBytes;
+constexpr int kSmemBytes = 5 * kTileBytes + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
+// Registers per thread: the CTA is launched with kLaunchRegs each (the whole register
+// file); the producer warpgroups hand kLaunchRegs - kProducerRegs each back and the
+// softmax warpgroups take the same amount, so the two sums match exactly (setmaxnreg).
+constexpr int kLaunchRegs = 65536 / kAttnThreads;  // 128
+constexpr int kProducerRegs = 112, kSoftmaxRegs = 2 * kLaunchRegs - kProducerRegs;
+static_assert(kSoftmaxThreads == kProducerThreads && kSoftmaxRegs <= 256 && kSoftmaxRegs % 8 == 0 &&
+                  kProducerRegs % 8 == 0 && kProducerRegs >= 24,
+              "register split must balance");
 constexpr uint64_t kWaitNs = 1000000000ull;  // give up on an mbarrier after 1 s
 constexpr float kRescaleLog2 = 8.0f;          // rescale O when the row max grows by > 2^8
 constexpr int kMaxSplits = 64;
@@ -138,16 +150,19 @@ __device__ __forceinline__ void mma_qk(uint32_t tmem_d, uint32_t q_base, uint32_
                              sw128_desc(k_base + kb * 16384 + s * 32), kb > 0 || s > 0);
 }
 
-// O (TMEM) (+)= P[128 x 128 keys] V[128 keys x 128]: P K-major, V row-major (key rows, the
-// MN-major B operand); key step t of 16 keys starts 2048 B (two 8-row groups) further.
-__device__ __forceinline__ void mma_pv(uint32_t tmem_d, uint32_t p_base, uint32_t v_base, bool accumulate)
+// O (TMEM) (+)= P[128 x 128 keys] V[128 keys x 128]: P in TMEM (row i in lane i, keys 2c
+// and 2c + 1 in the low and high halves of column c), V row-major in shared memory (key
+// rows, the MN-major B operand). Key step t of 16 keys: P columns 8t on, V 2048 B (two
+// 8-row groups) further.
+__device__ __forceinline__ void mma_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_base, bool accumulate)
 {
 #pragma unroll
-    for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-        for (int s = 0; s < 4; ++s)
-            mma_bf16<kIdescBmn>(tmem_d, sw128_desc(p_base + kb * 16384 + s * 32),
-                                sw128_mn_desc(v_base + (kb * 4 + s) * 2048), accumulate || kb > 0 || s > 0);
+    for (int t = 0; t < 8; ++t)
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                     ::"r"(tmem_d), "r"(tmem_p + 8 * t), "l"(sw128_mn_desc(v_base + t * 2048)), "r"(kIdescBmn),
+                     "r"(accumulate || t > 0 ? 1u : 0u)
+                     : "memory");
 }
 
 __device__ __forceinline__ void commit(uint32_t mbar)
@@ -217,18 +232,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32])
 #pragma unroll
     for (int i = 0; i < 32; ++i)
         v[i] = __uint_as_float(r[i]);
-}
-
-// 16 columns of this warp's 32 TMEM lanes, without the wait: the registers are valid
-// only after tmem_wait_ld() and must not be read before it.
-__device__ __forceinline__ void tmem_ld16_async(uint32_t addr, uint32_t (&r)[16])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-                   "=r"(r[15])
-                 : "r"(addr)
-                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -400,8 +403,6 @@ __device__ __forceinline__ float tile_row_max(uint32_t tS, int valid)
     return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), written
-// as bf16 to row r of P (K-major, 128B-swizzled); returns the fp32 sum of p.
 // max(a, b, c) in one instruction (sm_100).
 __device__ __forceinline__ float max3(float a, float b, float c)
 {
@@ -410,24 +411,26 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return d;
 }
 
-// 16 columns (chunk c) of the row: p into P, sums into the packed accumulators; with
-// TRACK also the max of the raw scores into mt.
+// kW columns (chunk c) of the row: p as bf16 pairs into words c kW / 2 .. (c + 1) kW / 2 - 1
+// of P, sums into the packed accumulators; with TRACK also the max of the raw scores into
+// mt. The callers unroll over c, so P stays in registers.
+constexpr int kW = 8;  // columns per TMEM load of S
 template <bool MASK, bool TRACK>
-__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[16], int c, uint32_t sP, int r, int valid,
+__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[kW], int c, uint32_t (&P)[64], int valid,
                                           uint64_t sc2, uint64_t nm2, uint64_t& la, uint64_t& lb, float& mt)
 {
     const uint64_t one2 = f32x2_pack(1.0f, 1.0f);
-    uint32_t pw[8];
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
+    for (int i = 0; i < kW; i += 2) {
+        const int col = c * kW + i;
         const float s0 = __uint_as_float(sr[i]), s1 = __uint_as_float(sr[i + 1]);
         if (TRACK) {
             if (!MASK)
                 mt = max3(mt, s0, s1);
             else {
-                if (c * 16 + i < valid)
+                if (col < valid)
                     mt = fmaxf(mt, s0);
-                if (c * 16 + i + 1 < valid)
+                if (col + 1 < valid)
                     mt = fmaxf(mt, s1);
             }
         }
@@ -435,46 +438,54 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[16], int c, uint3
         f32x2_unpack(f32x2_fma(f32x2_pack(s0, s1), sc2, nm2), x0, x1);
         float p0 = ex2(x0), p1 = ex2(x1);
         if (MASK) {
-            if (c * 16 + i >= valid)
+            if (col >= valid)
                 p0 = 0.0f;
-            if (c * 16 + i + 1 >= valid)
+            if (col + 1 >= valid)
                 p1 = 0.0f;
         }
-        if ((i >> 1) & 1)
+        if ((col >> 1) & 1)
             lb = f32x2_fma(f32x2_pack(p0, p1), one2, lb);
         else
             la = f32x2_fma(f32x2_pack(p0, p1), one2, la);
-        pw[i >> 1] = bf16x2_from_f32(p1, p0);
+        P[col >> 1] = bf16x2_from_f32(p1, p0);
     }
-    const int kb = c >> 2, ch0 = (c & 3) * 2;
-    st_shared_v4(sP + sw128(r, kb, ch0), pw[0], pw[1], pw[2], pw[3]);
-    st_shared_v4(sP + sw128(r, kb, ch0 + 1), pw[4], pw[5], pw[6], pw[7]);
 }
 
-// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), written
-// as bf16 to row r of P (K-major, 128B-swizzled); returns the fp32 sum of p and, with
-// TRACK, the max of the raw scores in mt. The TMEM load of the next 16 columns is in
-// flight while the current ones are computed.
+// kW columns of this warp's 32 TMEM lanes, without the wait: the registers are valid
+// only after tmem_wait_ld() and must not be read before it.
+__device__ __forceinline__ void tmem_ldw_async(uint32_t addr, uint32_t (&r)[kW])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), as bf16
+// pairs into P (registers; word c holds keys 2c, 2c + 1); returns the fp32 sum of p and,
+// with TRACK, the max of the raw scores in mt. The TMEM load of the next kW columns is
+// in flight while the current ones are computed.
 template <bool MASK, bool TRACK>
-__device__ __forceinline__ float tile_row_exp(uint32_t tS, uint32_t sP, int r, int valid, float scale_log2, float m,
+__device__ __forceinline__ float tile_row_exp(uint32_t tS, uint32_t (&P)[64], int valid, float scale_log2, float m,
                                               float& mt)
 {
+    constexpr int kChunks = kBN / kW;
     const uint64_t sc2 = f32x2_pack(scale_log2, scale_log2), nm2 = f32x2_pack(-m, -m);
     uint64_t la = 0, lb = 0;  // two packed partial sums (+0.0 bit patterns)
-    uint32_t r0[16], r1[16];
+    uint32_t r0[kW], r1[kW];
     mt = -INFINITY;
-    tmem_ld16_async(tS, r0);
+    tmem_ldw_async(tS, r0);
     tmem_wait_ld();
-#pragma unroll 1
-    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int k = 0; k < kChunks / 2; ++k) {
         const int c = 2 * k;
-        tmem_ld16_async(tS + (c + 1) * 16, r1);
-        exp_chunk<MASK, TRACK>(r0, c, sP, r, valid, sc2, nm2, la, lb, mt);
+        tmem_ldw_async(tS + (c + 1) * kW, r1);
+        exp_chunk<MASK, TRACK>(r0, c, P, valid, sc2, nm2, la, lb, mt);
         tmem_wait_ld();
-        if (k < 3)
-            tmem_ld16_async(tS + (c + 2) * 16, r0);
-        exp_chunk<MASK, TRACK>(r1, c + 1, sP, r, valid, sc2, nm2, la, lb, mt);
-        if (k < 3)
+        if (k < kChunks / 2 - 1)
+            tmem_ldw_async(tS + (c + 2) * kW, r0);
+        exp_chunk<MASK, TRACK>(r1, c + 1, P, valid, sc2, nm2, la, lb, mt);
+        if (k < kChunks / 2 - 1)
             tmem_wait_ld();
     }
     float a0, a1, b0, b1;
@@ -484,11 +495,25 @@ __device__ __forceinline__ float tile_row_exp(uint32_t tS, uint32_t sP, int r, i
 }
 
 template <bool TRACK>
-__device__ __forceinline__ float row_exp(uint32_t tS, uint32_t sP, int r, int valid, float scale_log2, float m,
+__device__ __forceinline__ float row_exp(uint32_t tS, uint32_t (&P)[64], int valid, float scale_log2, float m,
                                          float& mt)
 {
-    return valid == kBN ? tile_row_exp<false, TRACK>(tS, sP, r, valid, scale_log2, m, mt)
-                        : tile_row_exp<true, TRACK>(tS, sP, r, valid, scale_log2, m, mt);
+    return valid == kBN ? tile_row_exp<false, TRACK>(tS, P, valid, scale_log2, m, mt)
+                        : tile_row_exp<true, TRACK>(tS, P, valid, scale_log2, m, mt);
+}
+
+// The row's P (64 words) into TMEM columns tP .. tP + 63 of this thread's lane.
+__device__ __forceinline__ void store_p(uint32_t tP, const uint32_t (&P)[64])
+{
+#pragma unroll
+    for (int c = 0; c < 64; c += 16)
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+                     "%15,%16};"
+                     ::"r"(tP + c), "r"(P[c]), "r"(P[c + 1]), "r"(P[c + 2]), "r"(P[c + 3]), "r"(P[c + 4]),
+                     "r"(P[c + 5]), "r"(P[c + 6]), "r"(P[c + 7]), "r"(P[c + 8]), "r"(P[c + 9]), "r"(P[c + 10]),
+                     "r"(P[c + 11]), "r"(P[c + 12]), "r"(P[c + 13]), "r"(P[c + 14]), "r"(P[c + 15])
+                     : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ kernels
@@ -556,6 +581,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
     const uint32_t tmem = tmem_base_s;
 
     if (tid < kSoftmaxThreads) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ---------------------------------------------------------------- softmax + MMA issue
         // Lane 0 of the warpgroup's first warp issues this query tile's MMAs: S_g(j+1) and
         // P_g V(j) follow its own softmax, which waits on them anyway.
@@ -563,7 +589,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
         if (g < n_qt) {
             const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
             const uint32_t tS = tmem + g * 128 + lane_off, tO = tmem + 256 + g * 128 + lane_off;
-            const uint32_t sQ = base + kOffQ + g * kTileBytes, sP = base + kOffP + g * kTileBytes;
+            const uint32_t sQ = base + kOffQ + g * kTileBytes;
             const uint32_t bS = bar(kSFull0 + g), bP = bar(kPFull0 + g), bO = bar(kODone0 + g);
             const bool issuer = r == 0;
             float m_run = -INFINITY, l_run = 0.0f;
@@ -593,29 +619,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                 }
                 float m_use, alpha, lt, mt;
                 bool need;
+                uint32_t P[64];
                 if (j == 0) {
                     // no reference yet: the row max first, then P
                     m_use = __fmul_rn(valid == kBN ? tile_row_max<false>(tS, valid) : tile_row_max<true>(tS, valid),
                                       a.scale_log2);
                     alpha = 0.0f;
                     need = true;
-                    lt = row_exp<false>(tS, sP, r, valid, a.scale_log2, m_use, mt);
+                    lt = row_exp<false>(tS, P, valid, a.scale_log2, m_use, mt);
                 } else {
                     // P against the reference max, tracking this tile's max; only when
                     // that max exceeds the reference by more than 2^8 (rare once the
                     // first tiles are seen) is P recomputed against it and O rescaled
-                    lt = row_exp<true>(tS, sP, r, valid, a.scale_log2, m_run, mt);
+                    lt = row_exp<true>(tS, P, valid, a.scale_log2, m_run, mt);
                     const float m_cand = fmaxf(m_run, __fmul_rn(mt, a.scale_log2));
                     need = m_cand > m_run + kRescaleLog2;
                     m_use = need ? m_cand : m_run;
                     alpha = need ? ex2(m_run - m_use) : 1.0f;
-                    if (__any_sync(0xFFFFFFFFu, need)) {
-                        const float lt2 = row_exp<false>(tS, sP, r, valid, a.scale_log2, m_use, mt);
-                        lt = need ? lt2 : lt;
-                    }
+                    // S is still whole in TMEM (P is not yet written over it); a row
+                    // that keeps its reference recomputes the same P and sum
+                    if (__any_sync(0xFFFFFFFFu, need))
+                        lt = row_exp<false>(tS, P, valid, a.scale_log2, m_use, mt);
                 }
                 l_run = __fmaf_rn(l_run, alpha, lt);
                 m_run = m_use;
+                store_p(tS, P);
                 // rescale O (the warp does it if any of its rows needs it)
                 if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
 #pragma unroll 1
@@ -628,7 +656,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                         tmem_st32(tO + c * 32, o);
                     }
                 }
-                fence_async_smem();
                 tc_before_sync();
                 mbar_arrive(bP);
                 if (issuer) {
@@ -636,7 +663,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                     ok = wait_phase(bP, j & 1) && wait_phase(bar(kVFull), j & 1);
                     if (ok) {
                         tc_after_sync();
-                        mma_pv(tmem + 256 + g * 128, sP, sV, j > 0);
+                        mma_pv(tmem + 256 + g * 128, tmem + g * 128, sV, j > 0);
                         commit(bO);
                         commit(bar(kVEmpty));
                         if (j + 1 < n_tiles) {
@@ -696,6 +723,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                 atomicExch(a.status, 1);
         }
     } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
         // ---------------------------------------------------------------- producers
         // K runs one key tile ahead of V (K has two stages): K(j+1) is stored before V(j),
         // so Q K^T of the next tile never waits for the V buffer, which P V(j-1) holds.
@@ -893,7 +921,18 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
     a.status = status;
 
-    cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    // setmaxnreg moves registers between warpgroups inside the CTA's launch allocation, so
+    // the split above balances only if the kernel is launched with exactly kLaunchRegs
+    // registers per thread; refuse to launch otherwise (an unbalanced split would wait
+    // for registers forever)
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel);
+    if (e != cudaSuccess)
+        return launched(e, "kvq_attention");
+    if (fa.numRegs != kLaunchRegs)
+        return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: kernel built with %d registers per thread, its register split needs %d",
+                    fa.numRegs, kLaunchRegs);
+    e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess)
         return launched(e, "kvq_attention");
     cudaLaunchAttribute attr[1];

@@ -14,25 +14,30 @@
 // workspace and combine_kernel merges them; the split count is chosen so the units fill
 // the SMs in whole waves.
 //
-// Roles inside the CTA (512 threads, 4 warps per SM sub-partition):
-//   warps 0-3, 4-7  softmax of query tile 0 / 1: thread t owns row t (TMEM lane t). Lane 0
-//                   of each warpgroup also issues that tile's tcgen05.mma and commits:
-//                   P V(j) and S(j+1) follow its own softmax, which waits on them anyway.
-//                   Warp 0 allocates and frees the TMEM.
+// Roles inside the CTA (544 threads, 17 warps):
+//   warps 0-3, 4-7  softmax of query tile 0 / 1: thread t owns row t (TMEM lane t). Per
+//                   key tile: the row max of S first, then p = 2^(s - m) written as bf16
+//                   into TMEM over the S columns already read. Warp 0 allocates and frees
+//                   the TMEM.
 //   warps 8-15      producers: load the packed K and V of a key tile (the next one while
 //                   the current is consumed, in registers) and dequantize it into
 //                   128B-swizzled shared memory as key rows: K is the K-major B operand of
-//                   Q K^T, V the MN-major B operand of P V.
+//                   Q K^T, V the MN-major B operand of P V. K and V have two stages each.
+//   warp 16         issues every tcgen05.mma (one elected lane) in the order S_0(0), S_1(0),
+//                   then per key tile j: P_0 V(j), S_0(j+1), P_1 V(j), S_1(j+1). Tile 1's S
+//                   thus lands half a period after tile 0's, and each tile's softmax runs
+//                   while the other tile's MMAs execute (the ping-pong of FlashAttention-4
+//                   on Blackwell); a tcgen05.mma blocks its issuer while the tensor pipe's
+//                   queue is full, which is why no softmax thread issues them.
 // TMEM (512 columns, fp32): S0, S1 at columns 0 and 128; O0, O1 at 256 and 384. P_g, the
 // bf16 probabilities, is written over the first 64 columns of S_g (two keys per column)
 // and is the A operand of P V straight from TMEM, so P never passes through shared
 // memory and P V reads only V there. S_g(j+1) overwrites P_g(j) only after P V(j) has
 // read it: a thread's tcgen05.mma operations run in the order it issues them.
-// Each query tile's softmax overlaps the other tile's MMAs (the ping-pong of
-// FlashAttention-4 on Blackwell). The softmax keeps a reference row max and rescales O
-// only when the max grows by more than 2^8 (exact in real arithmetic: O and l share the
-// reference). Every wait is bounded (1 s); on a timeout the kernel records an error, lets
-// its MMAs drain, frees its TMEM and returns.
+// The softmax keeps a reference row max and rescales O only when the max grows by more
+// than 2^8 (exact in real arithmetic: O and l share the reference). Every wait is bounded
+// (1 s); on a timeout the kernel records an error, lets its MMAs drain, frees its TMEM
+// and returns.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -51,20 +56,23 @@ constexpr int kBN = 128;  // keys per tile
 constexpr int kD = 128;   // head_dim (the only one supported)
 constexpr int kSoftmaxThreads = kQT * 128;
 constexpr int kProducerThreads = 256;
-constexpr int kAttnThreads = kSoftmaxThreads + kProducerThreads;  // 512: 4 warps per SM sub-partition
-constexpr int kPieces = 4 * kBN / kProducerThreads;                 // 16-byte pieces per producer thread
+constexpr int kMmaWarp = (kSoftmaxThreads + kProducerThreads) / 32;  // warp 16 issues every MMA
+constexpr int kAttnThreads = kSoftmaxThreads + kProducerThreads + 32;  // 544: 17 warps
+constexpr int kPieces = 4 * kBN / kProducerThreads;                    // 16-byte pieces per producer thread
 constexpr int kTileBytes = 32768;  // one 128 x 128 bf16 operand
-// dynamic shared memory: Q0, Q1, K stages 0 and 1, V (each 1024-aligned)
+// dynamic shared memory: Q0, Q1, K stages 0 and 1, V stages 0 and 1 (each 1024-aligned)
 constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = 4 * kTileBytes;
-constexpr int kSmemBytes = 5 * kTileBytes + 1024;  // + alignment slack
+constexpr int kSmemBytes = 6 * kTileBytes + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
-// Registers per thread: the CTA is launched with kLaunchRegs each (the whole register
-// file); the producer warpgroups hand kLaunchRegs - kProducerRegs each back and the
-// softmax warpgroups take the same amount, so the two sums match exactly (setmaxnreg).
-constexpr int kLaunchRegs = 65536 / kAttnThreads;  // 128
-constexpr int kProducerRegs = 112, kSoftmaxRegs = 2 * kLaunchRegs - kProducerRegs;
-static_assert(kSoftmaxThreads == kProducerThreads && kSoftmaxRegs <= 256 && kSoftmaxRegs % 8 == 0 &&
-                  kProducerRegs % 8 == 0 && kProducerRegs >= 24,
+// Registers per thread. A sub-partition holds at most 16 K registers and five of the 17
+// warps share one, so the CTA is launched with kLaunchRegs = 96 each (16 K / (5 * 32),
+// rounded down to the allocation step of 8). The softmax warpgroups then hand
+// kLaunchRegs - kSoftmaxRegs each back and the producer warpgroups take the same amount
+// (setmaxnreg), so the two sums match exactly; the MMA warp keeps kLaunchRegs.
+constexpr int kLaunchRegs = 96;
+constexpr int kSoftmaxRegs = 80, kProducerRegs = 2 * kLaunchRegs - kSoftmaxRegs;
+static_assert(kSoftmaxThreads == kProducerThreads && kProducerRegs <= 256 && kSoftmaxRegs % 8 == 0 &&
+                  kProducerRegs % 8 == 0 && kSoftmaxRegs >= 24 && 5 * 32 * kLaunchRegs <= 16384,
               "register split must balance");
 constexpr uint64_t kWaitNs = 1000000000ull;  // give up on an mbarrier after 1 s
 constexpr float kRescaleLog2 = 8.0f;          // rescale O when the row max grows by > 2^8
@@ -74,8 +82,8 @@ constexpr uint64_t kPartialBytesPerRow = kD * 4 + 8;
 
 // mbarriers
 enum {
-    kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull, kVEmpty,
-    kSFull0, kSFull1, kPFull0, kPFull1, kODone0, kODone1, kDone0, kDone1,
+    kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull0, kVFull1, kVEmpty0, kVEmpty1,
+    kSFull0, kSFull1, kPFull0, kPFull1, kODone0, kODone1, kMmaDone,
     kNumBars
 };
 
@@ -130,14 +138,9 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr)
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
 constexpr uint32_t kIdescBmn = kIdesc | (1u << 16);
 
-template <uint32_t IDESC>
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, bool accumulate)
-{
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 ::"r"(tmem_d), "l"(a), "l"(b), "r"(IDESC), "r"(accumulate ? 1u : 0u)
-                 : "memory");
-}
+// The MMA warp's instructions, in elected-lane form: the whole warp runs them, converged,
+// and elect.sync picks the one lane that issues -- always the same lane, so its commits
+// track all of its MMAs.
 
 // S (TMEM) = Q[128 x 128] K[128 x 128]^T, both K-major in shared memory, as 8 MMAs of K = 16.
 __device__ __forceinline__ void mma_qk(uint32_t tmem_d, uint32_t q_base, uint32_t k_base)
@@ -146,8 +149,11 @@ __device__ __forceinline__ void mma_qk(uint32_t tmem_d, uint32_t q_base, uint32_
     for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            mma_bf16<kIdesc>(tmem_d, sw128_desc(q_base + kb * 16384 + s * 32),
-                             sw128_desc(k_base + kb * 16384 + s * 32), kb > 0 || s > 0);
+            asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                         ::"r"(tmem_d), "l"(sw128_desc(q_base + kb * 16384 + s * 32)),
+                         "l"(sw128_desc(k_base + kb * 16384 + s * 32)), "r"(kIdesc), "r"(kb > 0 || s > 0 ? 1u : 0u)
+                         : "memory");
 }
 
 // O (TMEM) (+)= P[128 x 128 keys] V[128 keys x 128]: P in TMEM (row i in lane i, keys 2c
@@ -158,16 +164,18 @@ __device__ __forceinline__ void mma_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_
 {
 #pragma unroll
     for (int t = 0; t < 8; ++t)
-        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                     "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
                      ::"r"(tmem_d), "r"(tmem_p + 8 * t), "l"(sw128_mn_desc(v_base + t * 2048)), "r"(kIdescBmn),
                      "r"(accumulate || t > 0 ? 1u : 0u)
                      : "memory");
 }
 
+// Arrive on mbar once every MMA the elected lane has issued so far is complete.
 __device__ __forceinline__ void commit(uint32_t mbar)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(mbar)
                  : "memory");
 }
 
@@ -385,24 +393,6 @@ __device__ __forceinline__ void store_pieces(const RawPieces& r, uint32_t valid,
 
 // ------------------------------------------------------------------ softmax pieces
 
-// Max of row S over the tile's valid keys (MASK: only the first `valid`), in four
-// independent chains.
-template <bool MASK>
-__device__ __forceinline__ float tile_row_max(uint32_t tS, int valid)
-{
-    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        float s[32];
-        tmem_ld32(tS + c * 32, s);
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (!MASK || c * 32 + i < valid)
-                m[i & 3] = fmaxf(m[i & 3], s[i]);
-    }
-    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-}
-
 // max(a, b, c) in one instruction (sm_100).
 __device__ __forceinline__ float max3(float a, float b, float c)
 {
@@ -411,31 +401,73 @@ __device__ __forceinline__ float max3(float a, float b, float c)
     return d;
 }
 
-// kW columns (chunk c) of the row: p as bf16 pairs into words c kW / 2 .. (c + 1) kW / 2 - 1
-// of P, sums into the packed accumulators; with TRACK also the max of the raw scores into
-// mt. The callers unroll over c, so P stays in registers.
-constexpr int kW = 8;  // columns per TMEM load of S
-template <bool MASK, bool TRACK>
-__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[kW], int c, uint32_t (&P)[64], int valid,
-                                          uint64_t sc2, uint64_t nm2, uint64_t& la, uint64_t& lb, float& mt)
+constexpr int kW = 16;  // columns of S per TMEM load
+
+// kW columns of this warp's 32 TMEM lanes, without the wait: the registers are valid
+// only after tmem_wait_ld() and must not be read before it.
+__device__ __forceinline__ void tmem_ldw_async(uint32_t addr, uint32_t (&r)[kW])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// Max of row S over the tile's valid keys (MASK: only the first `valid`), in two chains of
+// three-input max; the load of the next kW columns is in flight while the current ones
+// are reduced.
+template <bool MASK>
+__device__ __forceinline__ void max_chunk(const uint32_t (&sr)[kW], int c, int valid, float& m0, float& m1)
+{
+#pragma unroll
+    for (int i = 0; i < kW; i += 4) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            v[u] = !MASK || c * kW + i + u < valid ? __uint_as_float(sr[i + u]) : -INFINITY;
+        m0 = max3(m0, v[0], v[1]);
+        m1 = max3(m1, v[2], v[3]);
+    }
+}
+
+template <bool MASK>
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int valid)
+{
+    constexpr int kChunks = kBN / kW;
+    float m0 = -INFINITY, m1 = -INFINITY;
+    uint32_t r0[kW], r1[kW];
+    tmem_ldw_async(tS, r0);
+    tmem_wait_ld();
+#pragma unroll 1
+    for (int k = 0; k < kChunks / 2; ++k) {
+        const int c = 2 * k;
+        tmem_ldw_async(tS + (c + 1) * kW, r1);
+        max_chunk<MASK>(r0, c, valid, m0, m1);
+        tmem_wait_ld();
+        if (k < kChunks / 2 - 1)
+            tmem_ldw_async(tS + (c + 2) * kW, r0);
+        max_chunk<MASK>(r1, c + 1, valid, m0, m1);
+        if (k < kChunks / 2 - 1)
+            tmem_wait_ld();
+    }
+    return fmaxf(m0, m1);
+}
+
+// kW columns (chunk c) of the row: p = 2^(s * scale_log2 - m) (0 past `valid` when MASK),
+// summed into the packed accumulators and written as bf16 pairs to TMEM columns
+// tS + c kW / 2 on, which hold S columns this thread has already read.
+template <bool MASK>
+__device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[kW], int c, uint32_t tS, int valid, uint64_t sc2,
+                                          uint64_t nm2, uint64_t& la, uint64_t& lb)
 {
     const uint64_t one2 = f32x2_pack(1.0f, 1.0f);
+    uint32_t pw[kW / 2];
 #pragma unroll
     for (int i = 0; i < kW; i += 2) {
         const int col = c * kW + i;
-        const float s0 = __uint_as_float(sr[i]), s1 = __uint_as_float(sr[i + 1]);
-        if (TRACK) {
-            if (!MASK)
-                mt = max3(mt, s0, s1);
-            else {
-                if (col < valid)
-                    mt = fmaxf(mt, s0);
-                if (col + 1 < valid)
-                    mt = fmaxf(mt, s1);
-            }
-        }
         float x0, x1;
-        f32x2_unpack(f32x2_fma(f32x2_pack(s0, s1), sc2, nm2), x0, x1);
+        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2), x0, x1);
         float p0 = ex2(x0), p1 = ex2(x1);
         if (MASK) {
             if (col >= valid)
@@ -443,82 +475,53 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[kW], int c, uint3
             if (col + 1 >= valid)
                 p1 = 0.0f;
         }
-        if ((col >> 1) & 1)
+        if ((i >> 1) & 1)
             lb = f32x2_fma(f32x2_pack(p0, p1), one2, lb);
         else
             la = f32x2_fma(f32x2_pack(p0, p1), one2, la);
-        P[col >> 1] = bf16x2_from_f32(p1, p0);
+        pw[i >> 1] = bf16x2_from_f32(p1, p0);
     }
-}
-
-// kW columns of this warp's 32 TMEM lanes, without the wait: the registers are valid
-// only after tmem_wait_ld() and must not be read before it.
-__device__ __forceinline__ void tmem_ldw_async(uint32_t addr, uint32_t (&r)[kW])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-                 : "r"(addr)
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"r"(tS + c * (kW / 2)), "r"(pw[0]), "r"(pw[1]), "r"(pw[2]), "r"(pw[3]), "r"(pw[4]), "r"(pw[5]),
+                 "r"(pw[6]), "r"(pw[7])
                  : "memory");
 }
 
-// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), as bf16
-// pairs into P (registers; word c holds keys 2c, 2c + 1); returns the fp32 sum of p and,
-// with TRACK, the max of the raw scores in mt. The TMEM load of the next kW columns is
-// in flight while the current ones are computed.
-template <bool MASK, bool TRACK>
-__device__ __forceinline__ float tile_row_exp(uint32_t tS, uint32_t (&P)[64], int valid, float scale_log2, float m,
-                                              float& mt)
+// p = 2^(s * scale_log2 - m) for row S of the tile (0 past `valid` when MASK), written as
+// bf16 into the first 64 columns of S (word c holds keys 2c, 2c + 1); returns the fp32
+// sum of p. The TMEM load of the next kW columns is in flight while the current ones are
+// computed; a chunk's P lands on columns loaded before it.
+template <bool MASK>
+__device__ __forceinline__ float tile_row_exp(uint32_t tS, int valid, float scale_log2, float m)
 {
     constexpr int kChunks = kBN / kW;
     const uint64_t sc2 = f32x2_pack(scale_log2, scale_log2), nm2 = f32x2_pack(-m, -m);
     uint64_t la = 0, lb = 0;  // two packed partial sums (+0.0 bit patterns)
     uint32_t r0[kW], r1[kW];
-    mt = -INFINITY;
     tmem_ldw_async(tS, r0);
     tmem_wait_ld();
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < kChunks / 2; ++k) {
         const int c = 2 * k;
         tmem_ldw_async(tS + (c + 1) * kW, r1);
-        exp_chunk<MASK, TRACK>(r0, c, P, valid, sc2, nm2, la, lb, mt);
+        exp_chunk<MASK>(r0, c, tS, valid, sc2, nm2, la, lb);
         tmem_wait_ld();
         if (k < kChunks / 2 - 1)
             tmem_ldw_async(tS + (c + 2) * kW, r0);
-        exp_chunk<MASK, TRACK>(r1, c + 1, P, valid, sc2, nm2, la, lb, mt);
+        exp_chunk<MASK>(r1, c + 1, tS, valid, sc2, nm2, la, lb);
         if (k < kChunks / 2 - 1)
             tmem_wait_ld();
     }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     float a0, a1, b0, b1;
     f32x2_unpack(la, a0, a1);
     f32x2_unpack(lb, b0, b1);
     return __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(b0, b1));
 }
 
-template <bool TRACK>
-__device__ __forceinline__ float row_exp(uint32_t tS, uint32_t (&P)[64], int valid, float scale_log2, float m,
-                                         float& mt)
-{
-    return valid == kBN ? tile_row_exp<false, TRACK>(tS, P, valid, scale_log2, m, mt)
-                        : tile_row_exp<true, TRACK>(tS, P, valid, scale_log2, m, mt);
-}
-
-// The row's P (64 words) into TMEM columns tP .. tP + 63 of this thread's lane.
-__device__ __forceinline__ void store_p(uint32_t tP, const uint32_t (&P)[64])
-{
-#pragma unroll
-    for (int c = 0; c < 64; c += 16)
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-                     "%15,%16};"
-                     ::"r"(tP + c), "r"(P[c]), "r"(P[c + 1]), "r"(P[c + 2]), "r"(P[c + 3]), "r"(P[c + 4]),
-                     "r"(P[c + 5]), "r"(P[c + 6]), "r"(P[c + 7]), "r"(P[c + 8]), "r"(P[c + 9]), "r"(P[c + 10]),
-                     "r"(P[c + 11]), "r"(P[c + 12]), "r"(P[c + 13]), "r"(P[c + 14]), "r"(P[c + 15])
-                     : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ kernels
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnArgs a)
+__global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
 {
     pdl_begin();
     extern __shared__ uint8_t smem_raw[];
@@ -537,11 +540,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
     const uint32_t base = (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) + 1023u) & ~1023u;
     const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(&bars[0]));
     auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-    const uint32_t sV = base + kOffV;
     // key tile j lives in K stage j % 2; its barriers' phase is j / 2
     auto sK = [base](int j) { return base + kOffK + static_cast<uint32_t>(j & 1) * kTileBytes; };
     auto kfull = [&bar](int j) { return bar(kKFull0 + (j & 1)); };
     auto kempty = [&bar](int j) { return bar(kKEmpty0 + (j & 1)); };
+    // and so does value tile j in V stage j % 2
+    auto sV = [base](int j) { return base + kOffV + static_cast<uint32_t>(j & 1) * kTileBytes; };
+    auto vfull = [&bar](int j) { return bar(kVFull0 + (j & 1)); };
+    auto vempty = [&bar](int j) { return bar(kVEmpty0 + (j & 1)); };
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -553,16 +559,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
     if (tid == 0) {
         for (int st = 0; st < 2; ++st) {
             mbar_init(bar(kKFull0 + st), kProducerThreads);
-            mbar_init(bar(kKEmpty0 + st), n_qt);  // one commit per active query tile's issuer
+            mbar_init(bar(kKEmpty0 + st), 1);  // one commit after the last MMA reading the stage
+            mbar_init(bar(kVFull0 + st), kProducerThreads);
+            mbar_init(bar(kVEmpty0 + st), 1);
         }
-        mbar_init(bar(kVFull), kProducerThreads);
-        mbar_init(bar(kVEmpty), n_qt);
         for (int g = 0; g < kQT; ++g) {
             mbar_init(bar(kSFull0 + g), 1);
             mbar_init(bar(kPFull0 + g), 128);
             mbar_init(bar(kODone0 + g), 1);
-            mbar_init(bar(kDone0 + g), 1);
         }
+        mbar_init(bar(kMmaDone), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // both query tiles -> shared memory (rows past n_q are zero)
@@ -578,31 +584,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
     tc_before_sync();
     __syncthreads();
     tc_after_sync();
-    const uint32_t tmem = tmem_base_s;
+    const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, tmem_base_s, 0);
 
     if (tid < kSoftmaxThreads) {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        // ---------------------------------------------------------------- softmax + MMA issue
-        // Lane 0 of the warpgroup's first warp issues this query tile's MMAs: S_g(j+1) and
-        // P_g V(j) follow its own softmax, which waits on them anyway.
-        const int g = tid >> 7, r = tid & 127;
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        // ---------------------------------------------------------------- softmax
+        const int g = __shfl_sync(0xFFFFFFFFu, tid >> 7, 0), r = tid & 127;
         if (g < n_qt) {
             const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
             const uint32_t tS = tmem + g * 128 + lane_off, tO = tmem + 256 + g * 128 + lane_off;
-            const uint32_t sQ = base + kOffQ + g * kTileBytes;
             const uint32_t bS = bar(kSFull0 + g), bP = bar(kPFull0 + g), bO = bar(kODone0 + g);
-            const bool issuer = r == 0;
             float m_run = -INFINITY, l_run = 0.0f;
             bool ok = true;
-            if (issuer && n_tiles > 0) {
-                ok = wait_phase(kfull(0), 0);
-                if (ok) {
-                    tc_after_sync();
-                    mma_qk(tmem + g * 128, sQ, sK(0));
-                    commit(bS);
-                    commit(kempty(0));
-                }
-            }
             for (int j = 0; ok && j < n_tiles; ++j) {
                 ok = warp_wait(bS, j & 1);
                 if (!ok)
@@ -610,42 +603,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                 tc_after_sync();
                 const int64_t key0 = static_cast<int64_t>(t_begin + j) * kBN;
                 const int valid = static_cast<int>(a.n_kv - key0 < kBN ? a.n_kv - key0 : kBN);
-                // P and O of this query tile are free once the previous P V is done
-                if (j > 0) {
+                // the row max first; the reference moves (and O is rescaled) only when the
+                // max exceeds it by more than 2^8, which is rare after the first tiles
+                const float mt = __fmul_rn(
+                    valid == kBN ? tile_row_max<false>(tS, valid) : tile_row_max<true>(tS, valid), a.scale_log2);
+                const float m_cand = j == 0 ? mt : fmaxf(m_run, mt);
+                const bool need = j == 0 || m_cand > m_run + kRescaleLog2;
+                const float m_use = need ? m_cand : m_run;
+                const float alpha = j == 0 ? 0.0f : (need ? ex2(m_run - m_use) : 1.0f);
+                // P over the S columns already read (S_g(j) was written after P V(j-1) had
+                // read P_g(j-1): both come from the MMA warp, in that order)
+                const float lt = valid == kBN ? tile_row_exp<false>(tS, valid, a.scale_log2, m_use)
+                                              : tile_row_exp<true>(tS, valid, a.scale_log2, m_use);
+                l_run = __fmaf_rn(l_run, alpha, lt);
+                m_run = m_use;
+                // rescale O (the warp does it if any of its rows needs it) once P V(j-1) is done
+                if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
                     ok = warp_wait(bO, (j - 1) & 1);
                     if (!ok)
                         break;
                     tc_after_sync();
-                }
-                float m_use, alpha, lt, mt;
-                bool need;
-                uint32_t P[64];
-                if (j == 0) {
-                    // no reference yet: the row max first, then P
-                    m_use = __fmul_rn(valid == kBN ? tile_row_max<false>(tS, valid) : tile_row_max<true>(tS, valid),
-                                      a.scale_log2);
-                    alpha = 0.0f;
-                    need = true;
-                    lt = row_exp<false>(tS, P, valid, a.scale_log2, m_use, mt);
-                } else {
-                    // P against the reference max, tracking this tile's max; only when
-                    // that max exceeds the reference by more than 2^8 (rare once the
-                    // first tiles are seen) is P recomputed against it and O rescaled
-                    lt = row_exp<true>(tS, P, valid, a.scale_log2, m_run, mt);
-                    const float m_cand = fmaxf(m_run, __fmul_rn(mt, a.scale_log2));
-                    need = m_cand > m_run + kRescaleLog2;
-                    m_use = need ? m_cand : m_run;
-                    alpha = need ? ex2(m_run - m_use) : 1.0f;
-                    // S is still whole in TMEM (P is not yet written over it); a row
-                    // that keeps its reference recomputes the same P and sum
-                    if (__any_sync(0xFFFFFFFFu, need))
-                        lt = row_exp<false>(tS, P, valid, a.scale_log2, m_use, mt);
-                }
-                l_run = __fmaf_rn(l_run, alpha, lt);
-                m_run = m_use;
-                store_p(tS, P);
-                // rescale O (the warp does it if any of its rows needs it)
-                if (j > 0 && __any_sync(0xFFFFFFFFu, need)) {
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         float o[32];
@@ -658,26 +635,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                 }
                 tc_before_sync();
                 mbar_arrive(bP);
-                if (issuer) {
-                    // O_g += P_g V(j), then S_g(j+1) = Q_g K(j+1)^T
-                    ok = wait_phase(bP, j & 1) && wait_phase(bar(kVFull), j & 1);
-                    if (ok) {
-                        tc_after_sync();
-                        mma_pv(tmem + 256 + g * 128, tmem + g * 128, sV, j > 0);
-                        commit(bO);
-                        commit(bar(kVEmpty));
-                        if (j + 1 < n_tiles) {
-                            ok = wait_phase(kfull(j + 1), ((j + 1) >> 1) & 1);
-                            if (ok) {
-                                tc_after_sync();
-                                mma_qk(tmem + g * 128, sQ, sK(j + 1));
-                                commit(bS);
-                                commit(kempty(j + 1));
-                            }
-                        }
-                    }
-                }
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
             }
             if (ok && n_tiles > 0) {
                 ok = warp_wait(bO, (n_tiles - 1) & 1);
@@ -714,21 +671,64 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                         a.part_ml[prow] = make_float2(m_run, l_run);
                 }
             }
-            if (issuer) {
-                commit(bar(kDone0 + g));  // completes once every MMA this thread issued has
-                if (!wait_phase(bar(kDone0 + g), 0))
-                    ok = false;
-            }
             if (!ok && lane == 0)
                 atomicExch(a.status, 1);
         }
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------------------- MMA issue
+        const uint32_t sQ0 = base + kOffQ, sQ1 = base + kOffQ + kTileBytes;
+        bool ok = true;
+        if (n_tiles > 0) {
+            ok = warp_wait(kfull(0), 0);
+            if (ok) {
+                tc_after_sync();
+                mma_qk(tmem, sQ0, sK(0));
+                commit(bar(kSFull0));
+                if (n_qt == 2) {
+                    mma_qk(tmem + 128, sQ1, sK(0));
+                    commit(bar(kSFull1));
+                }
+                commit(kempty(0));
+            }
+        }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            for (int g = 0; g < n_qt; ++g) {
+                // O_g += P_g V(j), then S_g(j+1) = Q_g K(j+1)^T
+                ok = warp_wait(bar(kPFull0 + g), j & 1) && (g > 0 || warp_wait(vfull(j), (j >> 1) & 1));
+                if (!ok)
+                    break;
+                tc_after_sync();
+                mma_pv(tmem + 256 + g * 128, tmem + g * 128, sV(j), j > 0);
+                commit(bar(kODone0 + g));
+                if (g == n_qt - 1)
+                    commit(vempty(j));
+                if (j + 1 < n_tiles) {
+                    if (g == 0) {
+                        ok = warp_wait(kfull(j + 1), ((j + 1) >> 1) & 1);
+                        if (!ok)
+                            break;
+                        tc_after_sync();
+                    }
+                    mma_qk(tmem + g * 128, g == 0 ? sQ0 : sQ1, sK(j + 1));
+                    commit(bar(kSFull0 + g));
+                    if (g == n_qt - 1)
+                        commit(kempty(j + 1));
+                }
+            }
+        }
+        commit(bar(kMmaDone));  // completes once every MMA issued has
+        if (!warp_wait(bar(kMmaDone), 0))
+            ok = false;
+        if (!ok && lane == 0)
+            atomicExch(a.status, 1);
     } else {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
         // ---------------------------------------------------------------- producers
-        // K runs one key tile ahead of V (K has two stages): K(j+1) is stored before V(j),
-        // so Q K^T of the next tile never waits for the V buffer, which P V(j-1) holds.
-        // Each tensor's raw pieces are refilled right after its tile is stored, so the
-        // loads land while the other tensor is dequantized and the barriers are awaited.
+        // K runs one key tile ahead of V: K(j+1) is stored before V(j), the order in which
+        // the MMA warp consumes them (P_0 V(j) comes before S_0(j+1) but the V stage it
+        // needs was freed a tile earlier). Each tensor's raw pieces are refilled right
+        // after its tile is stored, so the loads land while the other tensor is
+        // dequantized and the barriers are awaited.
         const int p = tid - kSoftmaxThreads;
         auto key0_of = [&](int j) { return static_cast<int64_t>(t_begin + j) * kBN; };
         RawPieces rk, rv;
@@ -753,11 +753,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attention_kernel(const AttnAr
                 if (j + 2 < n_tiles)
                     load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(j + 2), p, rk);
             }
-            if (j > 0 && !(ok = wait_phase(bar(kVEmpty), (j - 1) & 1)))
+            // stage j % 2 was last read by the P V MMAs of value tile j - 2
+            if (j > 1 && !(ok = wait_phase(vempty(j), ((j >> 1) - 1) & 1)))
                 break;
-            store_pieces(rv, valid_pieces(a, key0_of(j), p), p, sV);
+            store_pieces(rv, valid_pieces(a, key0_of(j), p), p, sV(j));
             fence_async_smem();
-            mbar_arrive(bar(kVFull));
+            mbar_arrive(vfull(j));
             if (j + 1 < n_tiles)
                 load_pieces(a.vp, a.vs, a.va, a, h, key0_of(j + 1), p, rv);
         }

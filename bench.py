@@ -48,16 +48,23 @@ B_DEQUANT = 2.5625  # 0.5625 B read + bf16 written, per element
 L2_BYTES = 126 * 2 ** 20
 
 
-def kernel_source_sha256() -> str:
-    """SHA-256 of the measured kernels' code, comments and whitespace left out (the
-    profiles stay valid across comment edits, not across code changes)."""
+# The sources each traffic entry's counters depend on: an entry stays valid across edits of
+# other kernels and of comments, not across code changes of its own kernel.
+TRAFFIC_SOURCES = {
+    "codec": ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
+              "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"),
+    "attention": ("nvfp4_kv_cache_kvq_b200/csrc/kvq_attention.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
+                  "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"),
+}
+
+
+def kernel_source_sha256(group: str) -> str:
+    """SHA-256 of the code of one group of kernel sources, comments and whitespace left out."""
     import hashlib
     import re
 
     h = hashlib.sha256()
-    for rel in ("nvfp4_kv_cache_kvq_b200/csrc/kvq.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_rtn.cu",
-                "nvfp4_kv_cache_kvq_b200/csrc/kvq_attention.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
-                "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"):
+    for rel in TRAFFIC_SOURCES[group]:
         with open(os.path.join(ROOT, rel)) as f:
             src = f.read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)  # block comments
@@ -69,12 +76,12 @@ def kernel_source_sha256() -> str:
 def _traffic_entry(kind: str):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            t = json.load(f)
+            k = json.load(f).get("kernels", {}).get(kind)
     except Exception:
         return None
-    if t.get("source_sha256") != kernel_source_sha256():
+    if k is None or k.get("sources") not in TRAFFIC_SOURCES:
         return None
-    return t.get("kernels", {}).get(kind)
+    return k if k.get("source_sha256") == kernel_source_sha256(k["sources"]) else None
 
 
 def measured_traffic(kind: str):

@@ -414,45 +414,63 @@ __device__ __forceinline__ void tmem_ldw_async(uint32_t addr, uint32_t (&r)[kW])
                  : "memory");
 }
 
-// Max of row S over the tile's valid keys (MASK: only the first `valid`), in two chains of
-// three-input max; the load of the next kW columns is in flight while the current ones
-// are reduced.
-template <bool MASK>
-__device__ __forceinline__ void max_chunk(const uint32_t (&sr)[kW], int c, int valid, float& m0, float& m1)
-{
-#pragma unroll
-    for (int i = 0; i < kW; i += 4) {
-        float v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            v[u] = !MASK || c * kW + i + u < valid ? __uint_as_float(sr[i + u]) : -INFINITY;
-        m0 = max3(m0, v[0], v[1]);
-        m1 = max3(m1, v[2], v[3]);
-    }
-}
-
+// Max of row S over the tile's valid keys (MASK: only the first `valid`): four loads of 32
+// columns, each reduced in four independent chains of three-input max.
 template <bool MASK>
 __device__ __forceinline__ float tile_row_max(uint32_t tS, int valid)
 {
-    constexpr int kChunks = kBN / kW;
-    float m0 = -INFINITY, m1 = -INFINITY;
-    uint32_t r0[kW], r1[kW];
-    tmem_ldw_async(tS, r0);
-    tmem_wait_ld();
+    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-    for (int k = 0; k < kChunks / 2; ++k) {
-        const int c = 2 * k;
-        tmem_ldw_async(tS + (c + 1) * kW, r1);
-        max_chunk<MASK>(r0, c, valid, m0, m1);
-        tmem_wait_ld();
-        if (k < kChunks / 2 - 1)
-            tmem_ldw_async(tS + (c + 2) * kW, r0);
-        max_chunk<MASK>(r1, c + 1, valid, m0, m1);
-        if (k < kChunks / 2 - 1)
-            tmem_wait_ld();
+    for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tS + c * 32, v);
+        if (MASK) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                v[i] = c * 32 + i < valid ? v[i] : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+            m[0] = max3(m[0], v[i], v[i + 1]);
+            m[1] = max3(m[1], v[i + 2], v[i + 3]);
+            m[2] = max3(m[2], v[i + 4], v[i + 5]);
+            m[3] = max3(m[3], v[i + 6], v[i + 7]);
+        }
     }
-    return fmaxf(m0, m1);
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
+
+// 2^x for a pair of fp32 on the FMA pipe, for part of the softmax's exponentials (the ex2
+// unit takes the rest; FlashAttention-4 on Blackwell splits them the same way, since one
+// ex2 unit per sub-partition sets the softmax's pace). Range reduction after W. J. Cody
+// and W. Waite, "Software Manual for the Elementary Functions" (1980): x = n + f with n =
+// round(x) (adding 1.5 * 2^23 rounds to an integer and leaves n in the low mantissa bits)
+// and f in [-1/2, 1/2]; 2^f by a cubic fitted here to the relative error of 2^f on
+// [-1/2, 1/2] (iterated weighted least squares; max relative error 1.43e-4, far under
+// the 2^-9 of P's bf16 rounding); 2^n by adding n to the exponent field. x is clamped at
+// -125, so the result stays a normal number.
+__device__ __forceinline__ uint64_t exp2_poly(uint64_t x2)
+{
+    float x0, x1;
+    f32x2_unpack(x2, x0, x1);
+    const uint64_t x = f32x2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+    const uint64_t one2 = f32x2_pack(1.0f, 1.0f);
+    const uint64_t t = f32x2_fma(x, one2, f32x2_pack(12582912.0f, 12582912.0f));
+    const uint64_t n = f32x2_fma(t, one2, f32x2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f32x2_fma(n, f32x2_pack(-1.0f, -1.0f), x);
+    uint64_t p = f32x2_fma(f32x2_pack(0.055453190757429514f, 0.055453190757429514f), f,
+                           f32x2_pack(0.24236350527675452f, 0.24236350527675452f));
+    p = f32x2_fma(p, f, f32x2_pack(0.6931914699126007f, 0.6931914699126007f));
+    p = f32x2_fma(p, f, f32x2_pack(0.9999423493565059f, 0.9999423493565059f));
+    float p0, p1, t0, t1;
+    f32x2_unpack(p, p0, p1);
+    f32x2_unpack(t, t0, t1);
+    return f32x2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                      __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// Pairs of each kW-column chunk whose exponentials go to exp2_poly (bit i: pair i).
+constexpr uint32_t kPolyPairs = 0x88;
 
 // kW columns (chunk c) of the row: p = 2^(s * scale_log2 - m) (0 past `valid` when MASK),
 // summed into the packed accumulators and written as bf16 pairs to TMEM columns
@@ -466,9 +484,16 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&sr)[kW], int c, uint3
 #pragma unroll
     for (int i = 0; i < kW; i += 2) {
         const int col = c * kW + i;
-        float x0, x1;
-        f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2), x0, x1);
-        float p0 = ex2(x0), p1 = ex2(x1);
+        const uint64_t x2 = f32x2_fma(f32x2_pack(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
+        float p0, p1;
+        if ((kPolyPairs >> (i >> 1)) & 1) {
+            f32x2_unpack(exp2_poly(x2), p0, p1);
+        } else {
+            float x0, x1;
+            f32x2_unpack(x2, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+        }
         if (MASK) {
             if (col >= valid)
                 p0 = 0.0f;

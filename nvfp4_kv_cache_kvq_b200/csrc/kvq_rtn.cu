@@ -11,9 +11,10 @@
 // four per byte (element 4j + k in bits 2k..2k+1). The declarations in include/kvq.h
 // state the layout and the arguments.
 //
-// Kernels: one 16-element block per thread, one 256-bit load or store per block, CTA-
-// contiguous tiles, batches of tensors, programmatic dependent launch -- the same
-// skeleton as the NVFP4 kernels.
+// Kernels: two 16-element blocks per thread (one when the buffers are not aligned for
+// the wider code and scale accesses), one 256-bit load or store per block, CTA-contiguous
+// tiles, batches of tensors, programmatic dependent launch -- the same skeleton as the
+// NVFP4 kernels.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -128,17 +129,32 @@ __device__ __forceinline__ void rtn_dequantize_block(const uint32_t (&cw)[2], ui
     }
 }
 
-template <int BITS>
+// BPT blocks per thread (1 or 2). With 2, a thread moves 2 * BITS * 2 bytes of codes and
+// 4 bytes of scales in one access each, which needs codes aligned to 4 * BITS bytes and
+// scales to 4 bytes (the host picks BPT = 1 otherwise); an odd last block is handled on
+// its own.
+template <int BITS, int BPT>
 __global__ void __launch_bounds__(kThreads) rtn_quantize_kernel(const RtnBatch B)
 {
     pdl_begin();
     const RtnTensor& T = B.t[blockIdx.y];
-    const uint64_t b = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const uint64_t b = (static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x) * BPT;
     if (b >= B.n_blocks)
         return;
-    uint32_t w[8], cw[2];
-    ld_nc_v8(static_cast<const char*>(T.x) + b * 32, w);
+    const char* x = static_cast<const char*>(T.x);
+    uint32_t w[8], cw[2], cw1[2];
+    ld_nc_v8(x + b * 32, w);
     const uint32_t sb = rtn_quantize_block<BITS>(w, cw);
+    if (BPT == 2 && b + 1 < B.n_blocks) {
+        ld_nc_v8(x + b * 32 + 32, w);
+        const uint32_t sb1 = rtn_quantize_block<BITS>(w, cw1);
+        if (BITS == 4)
+            st_v4(T.packed + b * 8, cw[0], cw[1], cw1[0], cw1[1]);
+        else
+            st_v2(T.packed + b * 4, cw[0], cw1[0]);
+        *reinterpret_cast<uint32_t*>(T.scales + b) = sb | (sb1 << 16);
+        return;
+    }
     if (BITS == 4)
         st_v2(T.packed + b * 8, cw[0], cw[1]);
     else
@@ -146,15 +162,36 @@ __global__ void __launch_bounds__(kThreads) rtn_quantize_kernel(const RtnBatch B
     T.scales[b] = static_cast<uint16_t>(sb);
 }
 
-template <int BITS>
+template <int BITS, int BPT>
 __global__ void __launch_bounds__(kThreads) rtn_dequantize_kernel(const RtnBatch B)
 {
     pdl_begin();
     const RtnTensor& T = B.t[blockIdx.y];
-    const uint64_t b = static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x;
+    const uint64_t b = (static_cast<uint64_t>(blockIdx.x) * kThreads + threadIdx.x) * BPT;
     if (b >= B.n_blocks)
         return;
-    uint32_t cw[2] = {0u, 0u};
+    char* y = static_cast<char*>(const_cast<void*>(T.x));
+    uint32_t cw[2] = {0u, 0u}, out[8];
+    if (BPT == 2 && b + 1 < B.n_blocks) {
+        uint32_t cw1[2] = {0u, 0u};
+        if (BITS == 4) {
+            const uint4 q = ld_nc_v4(T.packed + b * 8);
+            cw[0] = q.x;
+            cw[1] = q.y;
+            cw1[0] = q.z;
+            cw1[1] = q.w;
+        } else {
+            const uint2 q = ld_nc_v2(T.packed + b * 4);
+            cw[0] = q.x;
+            cw1[0] = q.y;
+        }
+        const uint32_t s2 = __ldg(reinterpret_cast<const uint32_t*>(T.scales + b));
+        rtn_dequantize_block<BITS>(cw, s2 & 0xFFFFu, out);
+        st_v8(y + b * 32, out);
+        rtn_dequantize_block<BITS>(cw1, s2 >> 16, out);
+        st_v8(y + b * 32 + 32, out);
+        return;
+    }
     if (BITS == 4) {
         const uint2 q = ld_nc_v2(T.packed + b * 8);
         cw[0] = q.x;
@@ -162,9 +199,16 @@ __global__ void __launch_bounds__(kThreads) rtn_dequantize_kernel(const RtnBatch
     } else {
         cw[0] = __ldg(reinterpret_cast<const uint32_t*>(T.packed + b * 4));
     }
-    uint32_t y[8];
-    rtn_dequantize_block<BITS>(cw, __ldg(T.scales + b), y);
-    st_v8(static_cast<char*>(const_cast<void*>(T.x)) + b * 32, y);
+    rtn_dequantize_block<BITS>(cw, __ldg(T.scales + b), out);
+    st_v8(y + b * 32, out);
+}
+
+template <int BITS, int BPT>
+cudaError_t launch_rtn(bool quantize, uint64_t n_blocks, int m, const RtnBatch& rb, cudaStream_t s)
+{
+    const dim3 grid(tiles((n_blocks + BPT - 1) / BPT), m);
+    return quantize ? launch(rtn_quantize_kernel<BITS, BPT>, grid, kThreads, s, rb)
+                    : launch(rtn_dequantize_kernel<BITS, BPT>, grid, kThreads, s, rb);
 }
 
 kvq_status rtn_impl(bool quantize, const void* const* xs, uint8_t* const* packed, uint16_t* const* scales,
@@ -190,20 +234,21 @@ kvq_status rtn_impl(bool quantize, const void* const* xs, uint8_t* const* packed
                         2 * bits);
     }
     const uint64_t n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
+    // two blocks per thread when every buffer allows the wider accesses
+    bool wide = true;
+    for (int i = 0; i < n; ++i)
+        wide = wide && aligned(packed[i], 4 * bits) && aligned(scales[i], 4);
     for (int base = 0; base < n; base += kMaxBatch) {
         const int m = n - base < kMaxBatch ? n - base : kMaxBatch;
         RtnBatch rb{};
         rb.n_blocks = n_blocks;
         for (int i = 0; i < m; ++i)
             rb.t[i] = RtnTensor{xs[base + i], packed[base + i], scales[base + i]};
-        const dim3 grid(tiles(n_blocks), m);
         cudaError_t e;
-        if (quantize)
-            e = bits == 4 ? launch(rtn_quantize_kernel<4>, grid, kThreads, s, rb)
-                          : launch(rtn_quantize_kernel<2>, grid, kThreads, s, rb);
+        if (bits == 4)
+            e = wide ? launch_rtn<4, 2>(quantize, n_blocks, m, rb, s) : launch_rtn<4, 1>(quantize, n_blocks, m, rb, s);
         else
-            e = bits == 4 ? launch(rtn_dequantize_kernel<4>, grid, kThreads, s, rb)
-                          : launch(rtn_dequantize_kernel<2>, grid, kThreads, s, rb);
+            e = wide ? launch_rtn<2, 2>(quantize, n_blocks, m, rb, s) : launch_rtn<2, 1>(quantize, n_blocks, m, rb, s);
         if ((st = launched(e, what)) != KVQ_OK)
             return st;
     }

@@ -79,6 +79,29 @@ def test_rtn_extremes_and_ragged(orc, nbits):
     check(orc, z, nbits, 128)
 
 
+@pytest.mark.parametrize("nbits", [4, 2])
+def test_rtn_narrow_path_for_offset_buffers(orc, nbits):
+    """Codes aligned to 2*bits bytes and scales to 2 bytes, but not to 4*bits and 4: the
+    launch falls back to one block per thread; the results must not change. An odd block
+    count also leaves the two-block path's last block alone."""
+    x = inputs.normal((21, 16), seed=5, device="cuda")
+    n = x.numel()
+    pbuf = torch.zeros(n * nbits // 8 + 2 * nbits, dtype=torch.uint8, device="cuda")
+    sbuf = torch.zeros(n // 16 + 1, dtype=torch.bfloat16, device="cuda")
+    p_off, s_off = pbuf[2 * nbits:], sbuf[1:]
+    assert p_off.data_ptr() % (4 * nbits) != 0 and s_off.data_ptr() % 4 != 0
+    p, s = kvq.kvq_rtn_quantize(x, nbits, 16, packed=p_off, scales=s_off)
+    ybuf = torch.zeros(n + 16, dtype=torch.bfloat16, device="cuda")
+    y = kvq.kvq_rtn_dequantize(p, s, nbits, 16, y=ybuf[16:])
+    torch.cuda.synchronize()
+    pe, se = orc.rtn_quantize(bits(x), 16, nbits)
+    assert_same(p.cpu().numpy(), pe, "codes")
+    assert_same(bits(s), se, "scales")
+    assert_same(bits(y), orc.rtn_dequantize(pe, se, 16, nbits), "dequant")
+    # the wide path on aligned buffers agrees
+    check(orc, x, nbits, 16)
+
+
 def test_rtn_k2_v4_batches(orc):
     """RTN_K2_V4: keys with 2 bits, values with 4, one batched call per kind."""
     ks = [inputs.layer_kv(0, heads=2, tokens=100, device="cuda"), inputs.cache_kv(1, 0, heads=2, tokens=100, device="cuda")]

@@ -587,6 +587,60 @@ class Rtn(Sweep):
         return nbytes, time.perf_counter() - t0, f"first {m} of {self.tokens} rows, {reps} repetitions"
 
 
+class Layout:
+    """The blocked scale layout (the 128 x 4 tiles block-scaled MMA operands read) of the
+    scales of a quantized [T, 128] tensor: scales [T, 8] -> blocked and back."""
+    name = "layout"
+
+    def __init__(self, args, rank):
+        self.tokens, self.cols, self.D = args.tokens, 8, 128
+        self.rank = rank
+        self.n = self.tokens * self.cols  # scale bytes
+        self.flush = 3 * self.n < L2_BYTES * 4
+        self.config = {"workload": f"blocked scale layout: the [{self.tokens},8] e4m3 scales of a quantized "
+                                   f"[{self.tokens},128] N(0,1) tensor, to blocked and back",
+                       "model": "scale layout conversion (synthetic)", "global_batch": 1, "seq_len": self.tokens,
+                       "parallelism": "replica per GPU",
+                       "l2": "flushed between timed steps (256 MB write)" if self.flush else "inputs larger than L2"}
+
+    def setup(self, kvq, inputs, dev):
+        self.kvq = kvq
+        x = inputs.sweep(self.tokens, device=dev)
+        _, self.s, _ = kvq.kvq_quantize(x, self.D, "static_6")
+        del x
+        self.nb = kvq.kvq_blocked_scale_bytes(self.tokens, self.cols)
+        self.b = torch.empty(self.nb, dtype=torch.uint8, device=dev)
+        self.back = torch.empty_like(self.s)
+
+    def segments(self):
+        kvq, byts = self.kvq, float(self.n + self.nb)
+
+        def to():
+            kvq.kvq_scales_to_blocked(self.s, self.tokens, self.cols, blocked=self.b)
+
+        def back():
+            kvq.kvq_scales_from_blocked(self.b, self.tokens, self.cols, scales=self.back)
+        return [Segment("to_blocked", to, 1, byts, h2d=(self.s,)), Segment("from_blocked", back, 1, byts)]
+
+    def d2h(self):
+        return [self.back]
+
+    def tokens_per_step(self):
+        return self.tokens
+
+    def oracle_sample(self, orc, inputs, budget_s):
+        m = min(self.tokens, 1 << 18)
+        xb = inputs.bits(inputs.sweep(self.tokens)[:m])
+        _, sc, _ = orc.quantize(xb, self.D, "static_6")
+        t0, nbytes, reps = time.perf_counter(), 0.0, 0
+        while reps < 1 or time.perf_counter() - t0 < min(budget_s, 5.0):
+            b = orc.scales_to_blocked(sc, m, self.cols)
+            orc.scales_from_blocked(b, m, self.cols)
+            nbytes += 2.0 * (m * self.cols + orc.blocked_bytes(m, self.cols))
+            reps += 1
+        return nbytes, time.perf_counter() - t0, f"scales of the first {m} of {self.tokens} rows, {reps} repetitions"
+
+
 class Recent:
     """The rollout under the RECENT2 cache policy of the Self-Forcing study (RTN_INT4
     RECENT2): every frame appends 1560 tokens per layer to 30 layers x {K, V} through
@@ -791,7 +845,7 @@ class Attention:
         return self.bytes_layer * m / self.tokens, dt, f"layer 0, {m} of {self.tokens} query rows"
 
 
-WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention, Recent)}
+WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention, Recent, Layout)}
 
 
 # ---------------------------------------------------------------------------- runner

@@ -356,8 +356,10 @@ kvq_status kvq_recent_read_batch(const kvq_recent_cache* caches, int32_t n_cache
  * at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
  *
  * kvq_scales_to_blocked    scales (device, rows*cols bytes) -> blocked (device,
- *                          kvq_blocked_scale_bytes bytes, 4-byte aligned, padding zeroed).
- * kvq_scales_from_blocked  the inverse; writes rows*cols bytes.
+ *                          kvq_blocked_scale_bytes bytes, 16-byte aligned, padding zeroed).
+ * kvq_scales_from_blocked  the inverse (blocked 16-byte aligned); writes rows*cols bytes.
+ * A blocked buffer that is not 16-byte aligned returns KVQ_ERR_MISALIGNED; the plain
+ * scales have no alignment requirement.
  * kvq_blocked_scale_bytes  host only: rows' * cols'.
  */
 kvq_status kvq_scales_to_blocked(const uint8_t* scales, int64_t rows, int32_t cols, uint8_t* blocked,

@@ -25,6 +25,35 @@ def test_blocked_round_trip(orc, rows, cols):
     assert_same(back.cpu().numpy(), m, "from_blocked")
 
 
+@pytest.mark.parametrize("cols", [4, 8])
+def test_blocked_byte_path_for_unaligned_scales(orc, cols):
+    """A plain buffer that is not 4-byte aligned takes the byte-by-byte path, in both
+    directions, with the same results."""
+    rows = 300
+    rng = np.random.default_rng(cols)
+    m = rng.integers(0, 256, rows * cols, dtype=np.uint8)
+    buf = torch.zeros(rows * cols + 1, dtype=torch.uint8, device="cuda")
+    d = buf[1:]
+    d.copy_(torch.from_numpy(m))
+    assert d.data_ptr() % 4 != 0
+    b = kvq.kvq_scales_to_blocked(d, rows, cols)
+    out = torch.zeros(rows * cols + 1, dtype=torch.uint8, device="cuda")
+    back = kvq.kvq_scales_from_blocked(b, rows, cols, scales=out[1:])
+    torch.cuda.synchronize()
+    assert_same(b.cpu().numpy(), orc.scales_to_blocked(m, rows, cols), "blocked")
+    assert_same(back.cpu().numpy(), m, "from_blocked")
+    assert int(out[0].item()) == 0
+
+
+def test_blocked_buffer_alignment_is_checked():
+    m = torch.zeros(128 * 8, dtype=torch.uint8, device="cuda")
+    buf = torch.zeros(kvq.kvq_blocked_scale_bytes(128, 8) + 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_scales_to_blocked(m, 128, 8, blocked=buf[4:4 + kvq.kvq_blocked_scale_bytes(128, 8)])
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_scales_from_blocked(buf[4:4 + kvq.kvq_blocked_scale_bytes(128, 8)], 128, 8)
+
+
 def test_blocked_scales_of_a_quantized_layer(orc):
     x = inputs.layer_kv(0, heads=3, tokens=777, device="cuda")
     _, scales, _ = kvq.kvq_quantize(x, 128, "mse")

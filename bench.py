@@ -55,6 +55,10 @@ TRAFFIC_SOURCES = {
               "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"),
     "attention": ("nvfp4_kv_cache_kvq_b200/csrc/kvq_attention.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
                   "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"),
+    "rtn": ("nvfp4_kv_cache_kvq_b200/csrc/kvq_rtn.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
+            "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"),
+    "layout": ("nvfp4_kv_cache_kvq_b200/csrc/kvq_layout.cu", "nvfp4_kv_cache_kvq_b200/csrc/kvq_device.cuh",
+               "nvfp4_kv_cache_kvq_b200/csrc/kvq_common.h"),
 }
 
 
@@ -589,7 +593,8 @@ class Rtn(Sweep):
 
 class Layout:
     """The blocked scale layout (the 128 x 4 tiles block-scaled MMA operands read) of the
-    scales of a quantized [T, 128] tensor: scales [T, 8] -> blocked and back."""
+    scales of a [T, 128] tensor: scales [T, 8] (seeded e4m3 codes; the conversion is a
+    permutation, so its cost does not depend on them) -> blocked and back."""
     name = "layout"
 
     def __init__(self, args, rank):
@@ -597,17 +602,15 @@ class Layout:
         self.rank = rank
         self.n = self.tokens * self.cols  # scale bytes
         self.flush = 3 * self.n < L2_BYTES * 4
-        self.config = {"workload": f"blocked scale layout: the [{self.tokens},8] e4m3 scales of a quantized "
-                                   f"[{self.tokens},128] N(0,1) tensor, to blocked and back",
+        self.config = {"workload": f"blocked scale layout: the [{self.tokens},8] e4m3 scales of a "
+                                   f"[{self.tokens},128] tensor, to blocked and back",
                        "model": "scale layout conversion (synthetic)", "global_batch": 1, "seq_len": self.tokens,
                        "parallelism": "replica per GPU",
                        "l2": "flushed between timed steps (256 MB write)" if self.flush else "inputs larger than L2"}
 
     def setup(self, kvq, inputs, dev):
         self.kvq = kvq
-        x = inputs.sweep(self.tokens, device=dev)
-        _, self.s, _ = kvq.kvq_quantize(x, self.D, "static_6")
-        del x
+        self.s = inputs.scale_codes(self.tokens, self.cols, self.tokens, device=dev)
         self.nb = kvq.kvq_blocked_scale_bytes(self.tokens, self.cols)
         self.b = torch.empty(self.nb, dtype=torch.uint8, device=dev)
         self.back = torch.empty_like(self.s)
@@ -630,8 +633,7 @@ class Layout:
 
     def oracle_sample(self, orc, inputs, budget_s):
         m = min(self.tokens, 1 << 18)
-        xb = inputs.bits(inputs.sweep(self.tokens)[:m])
-        _, sc, _ = orc.quantize(xb, self.D, "static_6")
+        sc = inputs.scale_codes(m, self.cols, self.tokens).numpy()
         t0, nbytes, reps = time.perf_counter(), 0.0, 0
         while reps < 1 or time.perf_counter() - t0 < min(budget_s, 5.0):
             b = orc.scales_to_blocked(sc, m, self.cols)
@@ -1085,8 +1087,10 @@ def main():
         per_elem = {"dequant": B_DEQUANT, "append": B_AMAX + B_QUANT, "quantize": B_AMAX + B_QUANT,
                     "quantize_amax_in": B_QUANT,
                     "roundtrip": B_AMAX + B_QUANT + 2.0, "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16,
-                    "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16}.get(dom)
-        tb = measured_traffic(dom) if per_elem else None
+                    "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16,
+                    "to_blocked": 2.0, "from_blocked": 2.0}.get(dom)  # layout: per scale byte
+        # the RTN codecs' traffic depends on the bit width: their entries carry it
+        tb = measured_traffic(f"{dom}_int{args.bits}" if dom.startswith("rtn_") else dom) if per_elem else None
         elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom] if per_elem else None
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",

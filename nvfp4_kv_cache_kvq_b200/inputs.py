@@ -101,6 +101,13 @@ def sweep(tokens: int, device="cpu") -> torch.Tensor:
     return normal((tokens, HEAD_DIM), tokens, device)
 
 
+def scale_codes(rows: int, cols: int, seed: int, device="cpu") -> torch.Tensor:
+    """uint8 [rows * cols] e4m3 scale codes, uniform over 0x30 .. 0x6F (block scales
+    2^-3 .. 2^4 times the tensor's global scale), seed `seed`."""
+    g = _gen(seed, device)
+    return torch.randint(0x30, 0x70, (rows * cols,), generator=g, device=device, dtype=torch.int32).to(torch.uint8)
+
+
 def bits(x: torch.Tensor):
     """The bf16 bit patterns of a tensor as a flat numpy uint16 array (host copy)."""
     return x.detach().contiguous().view(torch.int16).cpu().numpy().view("uint16").reshape(-1)

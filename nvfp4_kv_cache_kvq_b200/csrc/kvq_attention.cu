@@ -58,12 +58,28 @@ constexpr int kSoftmaxThreads = kQT * 128;
 constexpr int kProducerThreads = 256;
 constexpr int kMmaWarp = (kSoftmaxThreads + kProducerThreads) / 32;  // warp 16 issues every MMA
 constexpr int kAttnThreads = kSoftmaxThreads + kProducerThreads + 32;  // 544: 17 warps
-constexpr int kPieces = 4 * kBN / kProducerThreads;                    // 16-byte pieces per producer thread
 constexpr int kTileBytes = 32768;  // one 128 x 128 bf16 operand
-// dynamic shared memory: Q0, Q1, K stages 0 and 1, V stages 0 and 1 (each 1024-aligned)
-constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = 4 * kTileBytes;
-constexpr int kSmemBytes = 6 * kTileBytes + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
+
+// Shared-memory geometry of one CTA. Alone (PAIR false) a CTA holds whole K and V tiles;
+// in a CTA pair each holds half of every tile -- keys 64 rank .. + 63 of K, dims 64 rank
+// .. + 63 of V -- the halves a cta_group::2 MMA takes from each CTA as its B operand.
+// Layout: Q0, Q1, K stages 0 and 1, V stages 0 and 1, each 1024-aligned.
+template <bool PAIR>
+struct Geo {
+    static constexpr int kKRows = PAIR ? kBN / 2 : kBN;  // key rows of K
+    static constexpr int kVDims = PAIR ? kD / 2 : kD;    // dims of V
+    static constexpr int kKBlock = kKRows * 128;         // one 64-dim K-block of K: kKRows x 128 B
+    static constexpr int kKBytes = 2 * kKBlock;
+    static constexpr int kVBytes = kBN * kVDims * 2;
+    static constexpr int kOffQ = 0, kOffK = 2 * kTileBytes, kOffV = kOffK + 2 * kKBytes;
+    static constexpr int kSmemBytes = kOffV + 2 * kVBytes + 1024;  // + alignment slack
+    static constexpr int kKPieces = kKRows * 4 / kProducerThreads;   // 16-byte K pieces per producer thread
+    static constexpr int kVQuarters = kVDims / 32;                   // 32-dim quarters of V per key row
+    static constexpr int kVPieces = kBN * kVQuarters / kProducerThreads;
+    static constexpr int kRowsPerUnit = (PAIR ? 2 : 1) * kQT * kBM;  // query rows per CTA (pair)
+    static constexpr int kCtas = PAIR ? 2 : 1;
+};
 // Registers per thread. A sub-partition holds at most 16 K registers and five of the 17
 // warps share one, so the CTA is launched with kLaunchRegs = 96 each (16 K / (5 * 32),
 // rounded down to the allocation step of 8). The softmax warpgroups then hand
@@ -134,59 +150,113 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr)
 }
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate, bf16 A and B, A
-// K-major, M = 128, N = 128; B K-major (kIdesc) or MN-major (kIdescBmn, bit 16).
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
-constexpr uint32_t kIdescBmn = kIdesc | (1u << 16);
+// K-major, N = 128, M = 128 (one CTA) or 256 (a CTA pair); B K-major (kIdesc) or
+// MN-major (kIdescBmn, bit 16).
+template <bool PAIR>
+constexpr uint32_t kIdesc =
+    (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((static_cast<uint32_t>(PAIR ? 2 : 1) * kBM >> 4) << 24);
+template <bool PAIR>
+constexpr uint32_t kIdescBmn = kIdesc<PAIR> | (1u << 16);
 
 // The MMA warp's instructions, in elected-lane form: the whole warp runs them, converged,
 // and elect.sync picks the one lane that issues -- always the same lane, so its commits
-// track all of its MMAs.
+// track all of its MMAs. With PAIR they are the cta_group::2 forms, issued by CTA 0 of
+// the pair for both CTAs (no output lane masked), and commits arrive on both CTAs'
+// copies of the barrier.
 
 // S (TMEM) = Q[128 x 128] K[128 x 128]^T, both K-major in shared memory, as 8 MMAs of K = 16.
+template <bool PAIR>
 __device__ __forceinline__ void mma_qk(uint32_t tmem_d, uint32_t q_base, uint32_t k_base)
 {
 #pragma unroll
     for (int kb = 0; kb < 2; ++kb)
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-            asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
-                         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                         ::"r"(tmem_d), "l"(sw128_desc(q_base + kb * 16384 + s * 32)),
-                         "l"(sw128_desc(k_base + kb * 16384 + s * 32)), "r"(kIdesc), "r"(kb > 0 || s > 0 ? 1u : 0u)
-                         : "memory");
+        for (int s = 0; s < 4; ++s) {
+            const uint64_t ad = sw128_desc(q_base + kb * 16384 + s * 32);
+            const uint64_t bd = sw128_desc(k_base + kb * Geo<PAIR>::kKBlock + s * 32);
+            const uint32_t acc = kb > 0 || s > 0 ? 1u : 0u;
+            if (PAIR)
+                asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                             "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;"
+                             "\n\t}" ::"r"(tmem_d), "l"(ad), "l"(bd), "r"(kIdesc<PAIR>), "r"(acc), "r"(0u)
+                             : "memory");
+            else
+                asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                             "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                             ::"r"(tmem_d), "l"(ad), "l"(bd), "r"(kIdesc<PAIR>), "r"(acc)
+                             : "memory");
+        }
 }
 
 // O (TMEM) (+)= P[128 x 128 keys] V[128 keys x 128]: P in TMEM (row i in lane i, keys 2c
 // and 2c + 1 in the low and high halves of column c), V row-major in shared memory (key
 // rows, the MN-major B operand). Key step t of 16 keys: P columns 8t on, V 2048 B (two
 // 8-row groups) further.
+template <bool PAIR>
 __device__ __forceinline__ void mma_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_base, bool accumulate)
 {
 #pragma unroll
-    for (int t = 0; t < 8; ++t)
-        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
-                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-                     ::"r"(tmem_d), "r"(tmem_p + 8 * t), "l"(sw128_mn_desc(v_base + t * 2048)), "r"(kIdescBmn),
-                     "r"(accumulate || t > 0 ? 1u : 0u)
+    for (int t = 0; t < 8; ++t) {
+        const uint64_t bd = sw128_mn_desc(v_base + t * 2048);
+        const uint32_t acc = accumulate || t > 0 ? 1u : 0u;
+        if (PAIR)
+            asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                         "@e tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;"
+                         "\n\t}" ::"r"(tmem_d), "r"(tmem_p + 8 * t), "l"(bd), "r"(kIdescBmn<PAIR>), "r"(acc), "r"(0u)
+                         : "memory");
+        else
+            asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                         ::"r"(tmem_d), "r"(tmem_p + 8 * t), "l"(bd), "r"(kIdescBmn<PAIR>), "r"(acc)
+                         : "memory");
+    }
+}
+
+// Arrive on mbar once every MMA the elected lane has issued so far is complete (on both
+// CTAs' copies with PAIR).
+template <bool PAIR>
+__device__ __forceinline__ void commit(uint32_t mbar)
+{
+    if (PAIR)
+        asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                     "\n\t}" ::"r"(mbar), "h"(static_cast<uint16_t>(3))
+                     : "memory");
+    else
+        asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(mbar)
                      : "memory");
 }
 
-// Arrive on mbar once every MMA the elected lane has issued so far is complete.
-__device__ __forceinline__ void commit(uint32_t mbar)
+// `count` arrivals on the barrier at this offset of CTA 0 of the pair (with PAIR; a
+// peer-CTA arrive from CTA 1) or of this CTA. What the arrival publishes is ordered by
+// the callers' tcgen05 and async-proxy fences, as for any arrive.
+template <bool PAIR>
+__device__ __forceinline__ void arrive_count(uint32_t mbar, uint32_t count)
 {
-    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(mbar)
-                 : "memory");
+    if (PAIR)
+        asm volatile("{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, 0;\n\t"
+                     "mbarrier.arrive.shared::cluster.b64 _, [ra], %1;\n\t}" ::"r"(mbar), "r"(count)
+                     : "memory");
+    else
+        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t mbar)
-{
-    asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(mbar) : "memory");
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns()
@@ -322,73 +392,59 @@ __device__ __forceinline__ float prefetch_f32(const float* p)
     return v;
 }
 
-// A producer thread's share of one tensor's key tile: kPieces pieces, piece i = 16 bytes
-// (2 blocks) of the row of key (p / 4) + 64 i, quarter q = p % 4 of the row (dims 32 q ..
-// 32 q + 31). A warp's loads thus cover 8 whole 64-byte rows each. Nothing is computed
-// from the loaded values here (they are the prefetch of the next tile and must not stall
-// the thread): keys past n_kv load row 0 instead and are zeroed at dequantization by
-// `valid`, and gs = amax / 2688 is taken there too.
-struct RawPieces {
-    uint4 c[kPieces];       // codes
-    uint32_t sc[kPieces];   // scale-code pair (blocks 2q, 2q+1) in the low 16 bits
-    float amax[kPieces];    // chunk amax of the key
+// One 16-byte piece of a key row: two blocks (32 dims, quarter q of the row). Nothing is
+// computed from the loaded values here (they are the prefetch of the next tile and must
+// not stall the thread): a key past n_kv loads row 0 instead and is zeroed at
+// dequantization, where gs = amax / 2688 is taken too.
+struct RawPiece {
+    uint4 c;      // codes
+    uint32_t sc;  // the two blocks' scale codes in the low 16 bits
+    float amax;   // chunk amax of the key
 };
 
 __device__ __forceinline__ float global_scale(float amax) { return __fdiv_rn(amax, 2688.0f); }
 
 // Keys and chunk indices fit in 32 bits (a cache holds at most 2^36 elements, i.e. 2^29
 // rows of 128).
-__device__ __forceinline__ void load_pieces(const uint8_t* packed, const uint8_t* scales, const float* amax,
-                                            const AttnArgs& a, int h, int64_t key0, int p, RawPieces& r)
+__device__ __forceinline__ void load_piece(const uint8_t* packed, const uint8_t* scales, const float* amax,
+                                           const AttnArgs& a, int h, int64_t key, int q, RawPiece& r)
 {
-    const int q = p & 3;
-#pragma unroll
-    for (int i = 0; i < kPieces; ++i) {
-        int64_t key = key0 + (p >> 2) + (kBN / kPieces) * i;
-        key = key < a.n_kv ? key : 0;
-        const int64_t off = (key * a.heads + h) * 64 + 16 * q;
-        const uint32_t chunk = static_cast<uint32_t>(key) / static_cast<uint32_t>(a.tokens_per_chunk);
-        r.c[i] = prefetch_v4(packed + off);
-        r.sc[i] = prefetch_u16(scales + off / 8);
-        r.amax[i] = prefetch_f32(amax + chunk);
-    }
+    key = key < a.n_kv ? key : 0;
+    const int64_t off = (key * a.heads + h) * 64 + 16 * q;
+    const uint32_t chunk = static_cast<uint32_t>(key) / static_cast<uint32_t>(a.tokens_per_chunk);
+    r.c = prefetch_v4(packed + off);
+    r.sc = prefetch_u16(scales + off / 8);
+    r.amax = prefetch_f32(amax + chunk);
 }
 
-// Bit i set when piece i's key is below n_kv.
-__device__ __forceinline__ uint32_t valid_pieces(const AttnArgs& a, int64_t key0, int p)
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in 64-wide block `kb` of a
+// 128B-swizzled operand whose blocks hold `rows` rows (8-row groups of 1024 B, the chunk
+// index XOR-ed with row % 8).
+__device__ __forceinline__ uint32_t sw128r(int row, int kb, int chunk, int rows)
 {
-    uint32_t m = 0;
-#pragma unroll
-    for (int i = 0; i < kPieces; ++i)
-        m |= (key0 + (p >> 2) + (kBN / kPieces) * i < a.n_kv ? 1u : 0u) << i;
-    return m;
+    return kb * rows * 128 + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
-// The four pieces dequantized into their rows of a 128B-swizzled tile (K as the K-major
-// B operand of Q K^T, V as the MN-major B operand of P V: the same bytes); invalid keys
-// get gs = 0, i.e. zeros. Threads of quarters 2 and 3 store their two blocks in swapped
-// order, so the 8 threads of each shared-memory wavefront hit 8 different 16-byte bank
-// groups.
-__device__ __forceinline__ void store_pieces(const RawPieces& r, uint32_t valid, int p, uint32_t sT)
+// The piece dequantized (the dequant kernel's arithmetic) into row `row`, chunks ch0 ..
+// ch0 + 3 of block kb of a swizzled operand of `rows` rows per block (K as the K-major B
+// operand of Q K^T, V as the MN-major B operand of P V: the same bytes); a key past n_kv
+// gives zeros. With swap the two blocks are stored in the other order, so that threads
+// of neighbouring quarters hit different 16-byte bank groups of a shared-memory wavefront.
+__device__ __forceinline__ void store_piece(const RawPiece& r, bool valid, int row, int kb, int ch0, int rows,
+                                            bool swap, uint32_t sT)
 {
-    const int q = p & 3, kb = q >> 1, swap = q & 2;
-#pragma unroll
-    for (int i = 0; i < kPieces; ++i) {
-        const int row = (p >> 2) + (kBN / kPieces) * i;
-        const float gs = (valid >> i) & 1u ? global_scale(r.amax[i]) : 0.0f;
-        const float SA = block_scale(r.sc[i], swap ? 1 : 0, gs), SB = block_scale(r.sc[i], swap ? 0 : 1, gs);
-        const uint4 c = r.c[i];
-        uint32_t y0[4], y1[4], y2[4], y3[4];
-        dequant8(swap ? c.z : c.x, SA, y0);
-        dequant8(swap ? c.w : c.y, SA, y1);
-        dequant8(swap ? c.x : c.z, SB, y2);
-        dequant8(swap ? c.y : c.w, SB, y3);
-        const int ch = (q & 1) * 4;
-        st_shared_v4(sT + sw128(row, kb, ch + (0 ^ swap)), y0[0], y0[1], y0[2], y0[3]);
-        st_shared_v4(sT + sw128(row, kb, ch + (1 ^ swap)), y1[0], y1[1], y1[2], y1[3]);
-        st_shared_v4(sT + sw128(row, kb, ch + (2 ^ swap)), y2[0], y2[1], y2[2], y2[3]);
-        st_shared_v4(sT + sw128(row, kb, ch + (3 ^ swap)), y3[0], y3[1], y3[2], y3[3]);
-    }
+    const float gs = valid ? global_scale(r.amax) : 0.0f;
+    const float SA = block_scale(r.sc, swap ? 1 : 0, gs), SB = block_scale(r.sc, swap ? 0 : 1, gs);
+    const int s2 = swap ? 2 : 0;
+    uint32_t y[4];
+    dequant8(swap ? r.c.z : r.c.x, SA, y);
+    st_shared_v4(sT + sw128r(row, kb, ch0 + (0 ^ s2), rows), y[0], y[1], y[2], y[3]);
+    dequant8(swap ? r.c.w : r.c.y, SA, y);
+    st_shared_v4(sT + sw128r(row, kb, ch0 + (1 ^ s2), rows), y[0], y[1], y[2], y[3]);
+    dequant8(swap ? r.c.x : r.c.z, SB, y);
+    st_shared_v4(sT + sw128r(row, kb, ch0 + (2 ^ s2), rows), y[0], y[1], y[2], y[3]);
+    dequant8(swap ? r.c.y : r.c.w, SB, y);
+    st_shared_v4(sT + sw128r(row, kb, ch0 + (3 ^ s2), rows), y[0], y[1], y[2], y[3]);
 }
 
 // ------------------------------------------------------------------ softmax pieces
@@ -546,51 +602,68 @@ __device__ __forceinline__ float tile_row_exp(uint32_t tS, int valid, float scal
 
 // ------------------------------------------------------------------ kernels
 
+// PAIR: the kernel runs as clusters of two CTAs (x even, x odd) that share every K/V
+// tile and issue cta_group::2 MMAs (M = 256: query tile slot g is rows 512 u + 256 g ..
+// + 255 of the pair, CTA `rank` holding the 128 from 512 u + 256 g + 128 rank); else one
+// CTA per unit of 256 query rows (slot g: rows 256 u + 128 g .. + 127).
+template <bool PAIR>
 __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
 {
+    using G = Geo<PAIR>;
     pdl_begin();
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[kNumBars];
     __shared__ uint32_t tmem_base_s;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qp = blockIdx.x, split = blockIdx.y, h = blockIdx.z;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;  // CTA 0 of a pair issues the MMAs
+    const int unit = PAIR ? blockIdx.x >> 1 : blockIdx.x, split = blockIdx.y, h = blockIdx.z;
     const int t_begin = static_cast<int>(static_cast<int64_t>(split) * a.key_tiles / a.splits);
     const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * a.key_tiles / a.splits);
     const int n_tiles = t_end - t_begin;
-    const int64_t q0 = static_cast<int64_t>(qp) * (kQT * kBM);
-    const int n_qt = a.n_q - q0 > kBM ? 2 : 1;  // query tiles holding rows
+    const int64_t u0 = static_cast<int64_t>(unit) * G::kRowsPerUnit;   // first row of the unit
+    const int64_t q0 = u0 + rank * kBM;                                // this CTA's first row
+    constexpr int kSlotRows = G::kCtas * kBM;                          // rows between slots
+    const int n_qt = a.n_q - u0 > kSlotRows ? 2 : 1;                   // slots holding rows
     const int64_t H = a.heads;
 
     const uint32_t base = (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) + 1023u) & ~1023u;
     const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(&bars[0]));
     auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     // key tile j lives in K stage j % 2; its barriers' phase is j / 2
-    auto sK = [base](int j) { return base + kOffK + static_cast<uint32_t>(j & 1) * kTileBytes; };
+    auto sK = [base](int j) { return base + G::kOffK + static_cast<uint32_t>(j & 1) * G::kKBytes; };
     auto kfull = [&bar](int j) { return bar(kKFull0 + (j & 1)); };
     auto kempty = [&bar](int j) { return bar(kKEmpty0 + (j & 1)); };
     // and so does value tile j in V stage j % 2
-    auto sV = [base](int j) { return base + kOffV + static_cast<uint32_t>(j & 1) * kTileBytes; };
+    auto sV = [base](int j) { return base + G::kOffV + static_cast<uint32_t>(j & 1) * G::kVBytes; };
     auto vfull = [&bar](int j) { return bar(kVFull0 + (j & 1)); };
     auto vempty = [&bar](int j) { return bar(kVEmpty0 + (j & 1)); };
 
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         static_cast<uint32_t>(__cvta_generic_to_shared(&tmem_base_s))),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        // a pair allocates together: warp 0 of both CTAs, the same destination offset
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&tmem_base_s));
+        if (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     if (tid == 0) {
+        // the "full" barriers count arrivals from every producer / softmax thread of the
+        // pair (only CTA 0's copy is waited on); the others take one commit each
         for (int st = 0; st < 2; ++st) {
-            mbar_init(bar(kKFull0 + st), kProducerThreads);
+            mbar_init(bar(kKFull0 + st), G::kCtas * kProducerThreads);
             mbar_init(bar(kKEmpty0 + st), 1);  // one commit after the last MMA reading the stage
-            mbar_init(bar(kVFull0 + st), kProducerThreads);
+            mbar_init(bar(kVFull0 + st), G::kCtas * kProducerThreads);
             mbar_init(bar(kVEmpty0 + st), 1);
         }
         for (int g = 0; g < kQT; ++g) {
             mbar_init(bar(kSFull0 + g), 1);
-            mbar_init(bar(kPFull0 + g), 128);
+            mbar_init(bar(kPFull0 + g), G::kCtas * kBM);
             mbar_init(bar(kODone0 + g), 1);
         }
         mbar_init(bar(kMmaDone), 1);
@@ -599,15 +672,17 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
     // both query tiles -> shared memory (rows past n_q are zero)
     for (int i = tid; i < kQT * kBM * 16; i += kAttnThreads) {
         const int g = i >> 11, row = (i >> 4) & 127, kb = (i >> 3) & 1, ch = i & 7;
-        const int64_t qrow = q0 + g * kBM + row;
+        const int64_t qrow = q0 + g * kSlotRows + row;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (qrow < a.n_q)
             v = ld_nc_v4(a.q + (qrow * H + h) * kD + kb * 64 + ch * 8);
-        st_shared_v4(base + kOffQ + g * kTileBytes + sw128(row, kb, ch), v.x, v.y, v.z, v.w);
+        st_shared_v4(base + G::kOffQ + g * kTileBytes + sw128(row, kb, ch), v.x, v.y, v.z, v.w);
     }
     fence_async_smem();
     tc_before_sync();
     __syncthreads();
+    if (PAIR)
+        cluster_sync();  // both CTAs' barriers initialized and TMEM allocated before any peer access
     tc_after_sync();
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, tmem_base_s, 0);
 
@@ -659,13 +734,15 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
                     }
                 }
                 tc_before_sync();
-                mbar_arrive(bP);
+                __syncwarp();
+                if (lane == 0)
+                    arrive_count<PAIR>(bP, 32);
             }
             if (ok && n_tiles > 0) {
                 ok = warp_wait(bO, (n_tiles - 1) & 1);
                 if (ok) {
                     tc_after_sync();
-                    const int64_t qrow = q0 + g * kBM + r;
+                    const int64_t qrow = q0 + g * kSlotRows + r;
                     const bool has_row = qrow < a.n_q;
                     const int64_t prow = (static_cast<int64_t>(split) * a.n_q + qrow) * H + h;
                     const float inv_l = 1.0f / l_run;
@@ -701,49 +778,53 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         }
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issue
-        const uint32_t sQ0 = base + kOffQ, sQ1 = base + kOffQ + kTileBytes;
+        // (CTA 0 of a pair issues for both CTAs; CTA 1's MMA warp has nothing to do)
+        const uint32_t sQ0 = base + G::kOffQ, sQ1 = base + G::kOffQ + kTileBytes;
         bool ok = true;
-        if (n_tiles > 0) {
+        const int tiles = rank == 0 ? n_tiles : 0;
+        if (tiles > 0) {
             ok = warp_wait(kfull(0), 0);
             if (ok) {
                 tc_after_sync();
-                mma_qk(tmem, sQ0, sK(0));
-                commit(bar(kSFull0));
+                mma_qk<PAIR>(tmem, sQ0, sK(0));
+                commit<PAIR>(bar(kSFull0));
                 if (n_qt == 2) {
-                    mma_qk(tmem + 128, sQ1, sK(0));
-                    commit(bar(kSFull1));
+                    mma_qk<PAIR>(tmem + 128, sQ1, sK(0));
+                    commit<PAIR>(bar(kSFull1));
                 }
-                commit(kempty(0));
+                commit<PAIR>(kempty(0));
             }
         }
-        for (int j = 0; ok && j < n_tiles; ++j) {
+        for (int j = 0; ok && j < tiles; ++j) {
             for (int g = 0; g < n_qt; ++g) {
                 // O_g += P_g V(j), then S_g(j+1) = Q_g K(j+1)^T
                 ok = warp_wait(bar(kPFull0 + g), j & 1) && (g > 0 || warp_wait(vfull(j), (j >> 1) & 1));
                 if (!ok)
                     break;
                 tc_after_sync();
-                mma_pv(tmem + 256 + g * 128, tmem + g * 128, sV(j), j > 0);
-                commit(bar(kODone0 + g));
+                mma_pv<PAIR>(tmem + 256 + g * 128, tmem + g * 128, sV(j), j > 0);
+                commit<PAIR>(bar(kODone0 + g));
                 if (g == n_qt - 1)
-                    commit(vempty(j));
-                if (j + 1 < n_tiles) {
+                    commit<PAIR>(vempty(j));
+                if (j + 1 < tiles) {
                     if (g == 0) {
                         ok = warp_wait(kfull(j + 1), ((j + 1) >> 1) & 1);
                         if (!ok)
                             break;
                         tc_after_sync();
                     }
-                    mma_qk(tmem + g * 128, g == 0 ? sQ0 : sQ1, sK(j + 1));
-                    commit(bar(kSFull0 + g));
+                    mma_qk<PAIR>(tmem + g * 128, g == 0 ? sQ0 : sQ1, sK(j + 1));
+                    commit<PAIR>(bar(kSFull0 + g));
                     if (g == n_qt - 1)
-                        commit(kempty(j + 1));
+                        commit<PAIR>(kempty(j + 1));
                 }
             }
         }
-        commit(bar(kMmaDone));  // completes once every MMA issued has
-        if (!warp_wait(bar(kMmaDone), 0))
-            ok = false;
+        if (rank == 0) {
+            commit<PAIR>(bar(kMmaDone));  // completes once every MMA issued has
+            if (!warp_wait(bar(kMmaDone), 0))
+                ok = false;
+        }
         if (!ok && lane == 0)
             atomicExch(a.status, 1);
     } else {
@@ -753,47 +834,87 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         // the MMA warp consumes them (P_0 V(j) comes before S_0(j+1) but the V stage it
         // needs was freed a tile earlier). Each tensor's raw pieces are refilled right
         // after its tile is stored, so the loads land while the other tensor is
-        // dequantized and the barriers are awaited.
+        // dequantized and the barriers are awaited. Piece i of thread p: K row
+        // (p + 256 i) / 4 of this CTA's key rows, quarter p % 4; V key row (p + 256 i) /
+        // kVQuarters, quarter p % kVQuarters of this CTA's dims. A warp's arrivals are one
+        // arrive of 32 (on CTA 0's barrier with PAIR).
         const int p = tid - kSoftmaxThreads;
         auto key0_of = [&](int j) { return static_cast<int64_t>(t_begin + j) * kBN; };
-        RawPieces rk, rv;
+        const int k_q = p & 3, v_q = p % G::kVQuarters;
+        auto k_row = [&](int i) { return (p + kProducerThreads * i) >> 2; };
+        auto v_row = [&](int i) { return (p + kProducerThreads * i) / G::kVQuarters; };
+        auto k_key = [&](int j, int i) { return key0_of(j) + rank * (kBN - G::kKRows) + k_row(i); };
+        auto v_key = [&](int j, int i) { return key0_of(j) + v_row(i); };
+        RawPiece rk[G::kKPieces], rv[G::kVPieces];
+        auto load_k = [&](int j) {
+#pragma unroll
+            for (int i = 0; i < G::kKPieces; ++i)
+                load_piece(a.kp, a.ks, a.ka, a, h, k_key(j, i), k_q, rk[i]);
+        };
+        auto load_v = [&](int j) {
+#pragma unroll
+            for (int i = 0; i < G::kVPieces; ++i)
+                load_piece(a.vp, a.vs, a.va, a, h, v_key(j, i), v_q + static_cast<int>(rank) * G::kVQuarters, rv[i]);
+        };
+        auto put_k = [&](int j) {
+#pragma unroll
+            for (int i = 0; i < G::kKPieces; ++i)
+                store_piece(rk[i], k_key(j, i) < a.n_kv, k_row(i), k_q >> 1, (k_q & 1) * 4, G::kKRows, (k_q & 2) != 0,
+                            sK(j));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                arrive_count<PAIR>(kfull(j), 32);
+        };
+        auto put_v = [&](int j) {
+#pragma unroll
+            for (int i = 0; i < G::kVPieces; ++i)
+                store_piece(rv[i], v_key(j, i) < a.n_kv, v_row(i), v_q >> 1, (v_q & 1) * 4, kBN, (v_q & 2) != 0,
+                            sV(j));
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                arrive_count<PAIR>(vfull(j), 32);
+        };
         bool ok = true;
         if (n_tiles > 0) {
-            load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(0), p, rk);
-            load_pieces(a.vp, a.vs, a.va, a, h, key0_of(0), p, rv);
-            store_pieces(rk, valid_pieces(a, key0_of(0), p), p, sK(0));
-            fence_async_smem();
-            mbar_arrive(kfull(0));
+            load_k(0);
+            load_v(0);
+            put_k(0);
             if (n_tiles > 1)
-                load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(1), p, rk);
+                load_k(1);
         }
         for (int j = 0; j < n_tiles; ++j) {
             if (j + 1 < n_tiles) {
                 // stage (j+1) % 2 was last read by the S MMAs of key tile j - 1
                 if (j > 0 && !(ok = wait_phase(kempty(j + 1), (((j + 1) >> 1) - 1) & 1)))
                     break;
-                store_pieces(rk, valid_pieces(a, key0_of(j + 1), p), p, sK(j + 1));
-                fence_async_smem();
-                mbar_arrive(kfull(j + 1));
+                put_k(j + 1);
                 if (j + 2 < n_tiles)
-                    load_pieces(a.kp, a.ks, a.ka, a, h, key0_of(j + 2), p, rk);
+                    load_k(j + 2);
             }
             // stage j % 2 was last read by the P V MMAs of value tile j - 2
             if (j > 1 && !(ok = wait_phase(vempty(j), ((j >> 1) - 1) & 1)))
                 break;
-            store_pieces(rv, valid_pieces(a, key0_of(j), p), p, sV(j));
-            fence_async_smem();
-            mbar_arrive(vfull(j));
+            put_v(j);
             if (j + 1 < n_tiles)
-                load_pieces(a.vp, a.vs, a.va, a, h, key0_of(j + 1), p, rv);
+                load_v(j + 1);
         }
         if (!ok && lane == 0)
             atomicExch(a.status, 1);
     }
     tc_before_sync();
     __syncthreads();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    if (PAIR)
+        cluster_sync();  // CTA 0's MMAs, which write both CTAs' TMEM, are all complete
+    if (warp == 0) {
+        if (PAIR)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                         : "memory");
+    }
 }
 
 // Merge the per-split partial results of one (query, head) row per warp:
@@ -858,6 +979,118 @@ uint64_t partial_bytes(int splits, int32_t n_q, int32_t heads)
     return splits > 1 ? static_cast<uint64_t>(splits) * n_q * heads * kPartialBytesPerRow : 0;
 }
 
+bool cluster_launch_supported()
+{
+    int dev = 0, v = 0;
+    return cudaGetDevice(&dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&v, cudaDevAttrClusterLaunch, dev) == cudaSuccess && v != 0;
+}
+
+// The launch plan: the query rows split into at most two parts, each launched on its own
+// (CTA pairs or single CTAs) with its key splits, workspace region and combine. A pair's
+// steady state takes about 15/16 of the time per query row of a single CTA (its M = 256
+// MMAs occupy each SM 76 cycles against 95 for M = 128; measured 7 % faster at 1024 and
+// 2048 queries), but its unit is 512 rows against 256. In units of a single CTA's time
+// per key tile, all single costs 16 ceil(n / 256), all pairs 30 ceil(n / 512), and pairs
+// over the whole 512-row blocks with single CTAs for the rest 30 floor(n / 512) +
+// 16 ceil((n mod 512) / 256); the cheapest wins (ties to fewer launches). 1560 queries
+// take three pairs for 1536 rows and one single CTA for the last 24.
+struct AttnPart {
+    bool pair;
+    int32_t row0, rows;  // query rows [row0, row0 + rows)
+    int64_t units;
+    int splits;
+    uint64_t ws_offset;  // of its partials in the workspace
+};
+
+struct AttnPlan {
+    int n_parts;
+    AttnPart part[2];
+    uint64_t ws_bytes;
+};
+
+constexpr uint64_t kWsAlign = 256;
+
+void finish_plan(AttnPlan& pl, int32_t heads)
+{
+    uint64_t off = 0;
+    for (int i = 0; i < pl.n_parts; ++i) {
+        pl.part[i].ws_offset = off;
+        off += (partial_bytes(pl.part[i].splits, pl.part[i].rows, heads) + kWsAlign - 1) / kWsAlign * kWsAlign;
+    }
+    pl.ws_bytes = off;
+}
+
+AttnPlan plan_attention(int32_t n_q, int32_t heads, int64_t key_tiles)
+{
+    constexpr int32_t kSingleRows = Geo<false>::kRowsPerUnit, kPairRows = Geo<true>::kRowsPerUnit;
+    const int64_t cost_single = 16 * ((n_q + kSingleRows - 1) / kSingleRows);
+    const int64_t cost_pair = 30 * ((n_q + kPairRows - 1) / kPairRows);
+    const int32_t full_rows = n_q / kPairRows * kPairRows, rest = n_q - full_rows;
+    const int64_t cost_mixed = 30 * (full_rows / kPairRows) + 16 * ((rest + kSingleRows - 1) / kSingleRows);
+    const bool pairs_ok = cluster_launch_supported();
+    AttnPlan pl{};
+    auto part = [&](bool pair, int32_t row0, int32_t rows) {
+        const int32_t unit_rows = pair ? kPairRows : kSingleRows;
+        AttnPart pt{};
+        pt.pair = pair;
+        pt.row0 = row0;
+        pt.rows = rows;
+        pt.units = (rows + unit_rows - 1) / unit_rows;
+        const int sms = sm_count();
+        pt.splits = choose_splits(pt.units * heads, static_cast<int>(key_tiles), pair ? sms / 2 : sms);
+        return pt;
+    };
+    if (!pairs_ok || (cost_single <= cost_pair && cost_single <= cost_mixed)) {
+        pl.n_parts = 1;
+        pl.part[0] = part(false, 0, n_q);
+    } else if (rest == 0 || cost_pair <= cost_mixed || full_rows == 0) {
+        pl.n_parts = 1;
+        pl.part[0] = part(true, 0, n_q);
+    } else {
+        pl.n_parts = 2;
+        pl.part[0] = part(true, 0, full_rows);
+        pl.part[1] = part(false, full_rows, rest);
+    }
+    finish_plan(pl, heads);
+    return pl;
+}
+
+// Check the register count (setmaxnreg moves registers between warpgroups inside the
+// CTA's launch allocation, so the split balances only if the kernel is launched with
+// exactly kLaunchRegs registers per thread: refuse to launch otherwise, since an
+// unbalanced split would wait for registers forever), set the shared-memory size, launch.
+template <bool PAIR>
+kvq_status launch_attention(const AttnArgs& a, int64_t units, int splits, int heads, cudaStream_t stream)
+{
+    cudaFuncAttributes fa{};
+    cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel<PAIR>);
+    if (e != cudaSuccess)
+        return launched(e, "kvq_attention");
+    if (fa.numRegs != kLaunchRegs)
+        return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: kernel built with %d registers per thread, its register split needs %d",
+                    fa.numRegs, kLaunchRegs);
+    e = cudaFuncSetAttribute(attention_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<PAIR>::kSmemBytes);
+    if (e != cudaSuccess)
+        return launched(e, "kvq_attention");
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = PAIR ? 2 : 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(Geo<PAIR>::kCtas * units), static_cast<unsigned>(splits),
+                       static_cast<unsigned>(heads));
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = Geo<PAIR>::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = PAIR ? 2 : 1;
+    return launched(cudaLaunchKernelEx(&cfg, attention_kernel<PAIR>, a), "kvq_attention");
+}
+
 }  // namespace
 }  // namespace kvq
 
@@ -872,9 +1105,10 @@ kvq_status kvq_attention_workspace_bytes(int32_t n_queries, int32_t heads, int64
     *bytes = 0;
     if (n_queries == 0 || n_keys == 0)
         return ok();
-    const int key_tiles = static_cast<int>((n_keys + kBN - 1) / kBN);
-    const int64_t units = static_cast<int64_t>((n_queries + kQT * kBM - 1) / (kQT * kBM)) * heads;
-    *bytes = partial_bytes(choose_splits(units, key_tiles, sm_count()), n_queries, heads);
+    const int64_t key_tiles = (n_keys + kBN - 1) / kBN;
+    if (key_tiles > INT32_MAX)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_attention_workspace_bytes: too many keys");
+    *bytes = plan_attention(n_queries, heads, key_tiles).ws_bytes;
     return ok();
 }
 
@@ -918,69 +1152,66 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
         return fail(KVQ_ERR_INVALID_ARG, "kvq_attention: too many keys");
     if (static_cast<int64_t>(n_queries) * heads / (kCombineThreads / 32) >= INT32_MAX)
         return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: n_queries * heads too large");
-    const int64_t qpairs = (n_queries + kQT * kBM - 1) / (kQT * kBM);
-    int splits = choose_splits(qpairs * heads, static_cast<int>(key_tiles), sm_count());
-    while (splits > 1 && partial_bytes(splits, n_queries, heads) > workspace_bytes)
-        --splits;
-    if (splits > 1 && (workspace == nullptr || !aligned(workspace, 16)))
+    // a workspace smaller than the plan's takes fewer key splits, the larger split first
+    AttnPlan plan = plan_attention(n_queries, heads, key_tiles);
+    while (plan.ws_bytes > workspace_bytes) {
+        AttnPart& big = plan.n_parts == 2 && plan.part[1].splits > plan.part[0].splits ? plan.part[1] : plan.part[0];
+        if (big.splits <= 1)
+            break;
+        --big.splits;
+        finish_plan(plan, heads);
+    }
+    if (plan.ws_bytes > 0 && (workspace == nullptr || !aligned(workspace, 16)))
         return fail(KVQ_ERR_MISALIGNED, "kvq_attention: workspace must be 16-byte aligned");
 
-    AttnArgs a;
-    a.q = static_cast<const uint16_t*>(q);
-    a.o = static_cast<uint16_t*>(out);
-    a.part_o = static_cast<float*>(workspace);
-    a.part_ml = splits > 1 ? reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) +
-                                                       static_cast<uint64_t>(splits) * n_queries * heads * kD * 4)
-                           : nullptr;
-    a.kp = k_cache->packed;
-    a.ks = k_cache->scales;
-    a.ka = k_cache->amax;
-    a.vp = v_cache->packed;
-    a.vs = v_cache->scales;
-    a.va = v_cache->amax;
-    a.n_q = n_queries;
-    a.heads = heads;
-    a.splits = splits;
-    a.key_tiles = static_cast<int32_t>(key_tiles);
-    a.n_kv = n_keys;
-    a.tokens_per_chunk = k_cache->rows_per_chunk / heads;
-    a.scale_log2 = softmax_scale * 1.4426950408889634f;
-    a.status = status;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    for (int i = 0; i < plan.n_parts; ++i) {
+        const AttnPart& pt = plan.part[i];
+        const uint64_t row_off = static_cast<uint64_t>(pt.row0) * heads * kD;
+        float* part_ws = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pt.ws_offset);
+        AttnArgs a;
+        a.q = static_cast<const uint16_t*>(q) + row_off;
+        a.o = static_cast<uint16_t*>(out) + row_off;
+        a.part_o = pt.splits > 1 ? part_ws : nullptr;
+        a.part_ml = pt.splits > 1 ? reinterpret_cast<float2*>(part_ws + static_cast<uint64_t>(pt.splits) * pt.rows * heads * kD)
+                                  : nullptr;
+        a.kp = k_cache->packed;
+        a.ks = k_cache->scales;
+        a.ka = k_cache->amax;
+        a.vp = v_cache->packed;
+        a.vs = v_cache->scales;
+        a.va = v_cache->amax;
+        a.n_q = pt.rows;
+        a.heads = heads;
+        a.splits = pt.splits;
+        a.key_tiles = static_cast<int32_t>(key_tiles);
+        a.n_kv = n_keys;
+        a.tokens_per_chunk = k_cache->rows_per_chunk / heads;
+        a.scale_log2 = softmax_scale * 1.4426950408889634f;
+        a.status = status;
 
-    // setmaxnreg moves registers between warpgroups inside the CTA's launch allocation, so
-    // the split above balances only if the kernel is launched with exactly kLaunchRegs
-    // registers per thread; refuse to launch otherwise (an unbalanced split would wait
-    // for registers forever)
-    cudaFuncAttributes fa{};
-    cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel);
-    if (e != cudaSuccess)
-        return launched(e, "kvq_attention");
-    if (fa.numRegs != kLaunchRegs)
-        return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: kernel built with %d registers per thread, its register split needs %d",
-                    fa.numRegs, kLaunchRegs);
-    e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess)
-        return launched(e, "kvq_attention");
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(qpairs), static_cast<unsigned>(splits), static_cast<unsigned>(heads));
-    cfg.blockDim = dim3(kAttnThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    kvq_status st = launched(cudaLaunchKernelEx(&cfg, attention_kernel, a), "kvq_attention");
-    if (st != KVQ_OK || splits == 1)
-        return st == KVQ_OK ? ok() : st;
-    const int64_t rows = static_cast<int64_t>(n_queries) * heads;
-    const int64_t rows_per_cta = kCombineThreads / 32;
-    cfg.gridDim = dim3(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta));
-    cfg.blockDim = dim3(kCombineThreads);
-    cfg.dynamicSmemBytes = 0;
-    st = launched(cudaLaunchKernelEx(&cfg, combine_kernel, a), "kvq_attention (combine)");
-    return st == KVQ_OK ? ok() : st;
+        kvq_status st = pt.pair ? launch_attention<true>(a, pt.units, pt.splits, heads, s)
+                                : launch_attention<false>(a, pt.units, pt.splits, heads, s);
+        if (st != KVQ_OK)
+            return st;
+        if (pt.splits == 1)
+            continue;
+        const int64_t rows = static_cast<int64_t>(pt.rows) * heads;
+        const int64_t rows_per_cta = kCombineThreads / 32;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta));
+        cfg.blockDim = dim3(kCombineThreads);
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        st = launched(cudaLaunchKernelEx(&cfg, combine_kernel, a), "kvq_attention (combine)");
+        if (st != KVQ_OK)
+            return st;
+    }
+    return ok();
 }
 
 }  // extern "C"

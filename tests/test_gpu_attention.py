@@ -91,6 +91,9 @@ def _workspace(split):
     (257, 2, 129, 64, "static_4"),   # one key past a tile; a second query pair
     (64, 4, 1000, 100, "mse"),
     (600, 1, 2000, 300, "mse"),      # three query pairs, the last with one partial tile
+    # CTA pairs (cta_group::2) take these: 2 x 15/16 x ceil(n_q / 512) < ceil(n_q / 256)
+    (400, 2, 300, 100, "mse"),       # one pair; CTA 1's second slot holds 16 rows
+    (1024, 1, 385, 64, "static_6"),  # two full pairs, a partial last key tile
 ])
 def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rule, split):
     caches, ocs = _filled_caches(orc, heads, n_keys, tokens_per_chunk, rule, 100)
@@ -134,10 +137,12 @@ def test_attention_peaked_scores(orc):
 
 def test_workspace_size_and_split_agree():
     """The recommended workspace is 0 exactly when no split is used, and a split result
-    agrees with the unsplit one (both are checked against the oracle above)."""
+    agrees with the unsplit one (both are checked against the oracle above). 1560 queries
+    over 732 key tiles split the keys of every query row at least in two, in 256-byte
+    aligned regions (one per launch part)."""
     assert kvq.kvq_attention_workspace_bytes(1, 1, 1) == 0
     b = kvq.kvq_attention_workspace_bytes(1560, 12, 93600)
-    assert b > 0 and b % (1560 * 12 * (128 * 4 + 8)) == 0
+    assert b >= 2 * 1560 * 12 * (128 * 4 + 8) and b % 256 == 0
 
 
 def test_attention_rollout_shape_sampled(orc):

@@ -45,11 +45,12 @@ def test_noalloc_matches_attention_twice_in_a_row():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # the rollout's attention (1560 queries x 12 heads over 93,600 keys) needs about
-    # 68 MB of partials: beyond the 32 MiB built in, so the call is refused up front
-    assert kvq.kvq_attention_workspace_bytes(1560, 12, 93600) > 32 << 20
-    caches = _caches(12, 16, 16, 3)
-    q = torch.zeros((1560, 12, D), dtype=torch.bfloat16, device="cuda")
+    # 4096 queries x 32 heads over 93,600 keys split their keys at least in two: over
+    # 100 MB of partials, beyond the 32 MiB built in, so the call is refused up front
+    n_q, heads, n_keys = 4096, 32, 93600
+    assert kvq.kvq_attention_workspace_bytes(n_q, heads, n_keys) > 32 << 20
+    caches = _caches(heads, 16, 16, 3)
+    q = torch.zeros((n_q, heads, D), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(kvq.KvqError) as e:
-        kvq.kvq_attention_noalloc(q, caches[0], caches[1], 93600)
+        kvq.kvq_attention_noalloc(q, caches[0], caches[1], n_keys)
     assert e.value.status == 4 and "scratch" in str(e.value)

@@ -782,7 +782,8 @@ class Attention:
             for l in range(self.layers):
                 kvq.kvq_attention(self.q[l], self.caches[2 * l], self.caches[2 * l + 1], self.n_keys,
                                   out=self.o[l], workspace=self.ws, status=self.status)
-        launches = self.layers * (2 if self.ws.numel() else 1)  # attention (+ combine) per layer
+        # one or two attention launches per layer, each followed by a combine when it splits keys
+        launches = self.layers * kvq.kvq_attention_launches(self.tokens, self.heads, self.n_keys)
         seg = Segment("attention", attn, launches, self.layers * self.bytes_layer, h2d=(self.q,))
         seg.flops = self.layers * self.flops_layer
         return [seg]

@@ -235,11 +235,16 @@ kvq_status kvq_dequantize_cache_batch(const kvq_cache* caches, void* const* ys, 
  *                incomplete); never cleared by the call.
  * kvq_attention_workspace_bytes -- host only: that size for these sizes (0 when no split
  *   would be used).
+ * kvq_attention_launches -- host only: how many kernels one kvq_attention call of these
+ *   sizes launches on the current device when given that workspace (1 to 4: the query
+ *   rows run in one or two parts, on CTA pairs or single CTAs, each followed by a
+ *   combine kernel when it splits its keys); 0 for n_queries == 0.
  */
 kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
                          const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out, void* workspace,
                          uint64_t workspace_bytes, int* status, kvq_stream_t stream);
 kvq_status kvq_attention_workspace_bytes(int32_t n_queries, int32_t heads, int64_t n_keys, uint64_t* bytes);
+kvq_status kvq_attention_launches(int32_t n_queries, int32_t heads, int64_t n_keys, int32_t* launches);
 
 /*
  * kvq_attention_noalloc -- kvq_attention without a workspace argument, for callers that

@@ -74,6 +74,7 @@ def load() -> ctypes.CDLL:
         "kvq_dequantize_cache_batch": [CP, ctypes.POINTER(P), I32, I64, I64, P],
         "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, ctypes.c_uint64, P, P],
         "kvq_attention_workspace_bytes": [I32, I32, I64, U64P],
+        "kvq_attention_launches": [I32, I32, I64, ctypes.POINTER(ctypes.c_int32)],
         "kvq_attention_noalloc": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, P],
         "kvq_recent_append_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
         "kvq_recent_read_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
@@ -365,6 +366,13 @@ def kvq_attention_workspace_bytes(n_queries: int, heads: int, n_keys: int) -> in
     b = ctypes.c_uint64()
     _check(load().kvq_attention_workspace_bytes(int(n_queries), int(heads), int(n_keys), ctypes.byref(b)))
     return b.value
+
+
+def kvq_attention_launches(n_queries: int, heads: int, n_keys: int) -> int:
+    """Kernels one kvq_attention call of these sizes launches with the recommended workspace."""
+    n = ctypes.c_int32()
+    _check(load().kvq_attention_launches(int(n_queries), int(heads), int(n_keys), ctypes.byref(n)))
+    return n.value
 
 
 def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: int,

@@ -1112,6 +1112,22 @@ kvq_status kvq_attention_workspace_bytes(int32_t n_queries, int32_t heads, int64
     return ok();
 }
 
+kvq_status kvq_attention_launches(int32_t n_queries, int32_t heads, int64_t n_keys, int32_t* launches)
+{
+    if (launches == nullptr || n_queries < 0 || heads <= 0 || n_keys < 0)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_attention_launches: bad arguments");
+    *launches = 0;
+    if (n_queries == 0)
+        return ok();
+    const int64_t key_tiles = (n_keys + kBN - 1) / kBN;
+    if (key_tiles > INT32_MAX)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_attention_launches: too many keys");
+    const AttnPlan plan = plan_attention(n_queries, heads, key_tiles);
+    for (int i = 0; i < plan.n_parts; ++i)
+        *launches += plan.part[i].splits > 1 ? 2 : 1;
+    return ok();
+}
+
 kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
                          const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out, void* workspace,
                          uint64_t workspace_bytes, int* status, kvq_stream_t stream)

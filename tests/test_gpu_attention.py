@@ -145,6 +145,17 @@ def test_workspace_size_and_split_agree():
     assert b >= 2 * 1560 * 12 * (128 * 4 + 8) and b % 256 == 0
 
 
+def test_attention_launch_count():
+    """The launch plan as kvq_attention_launches reports it: 1560 queries run as CTA pairs
+    over 1536 rows and single CTAs over the last 24, each part splitting its keys (two
+    attention launches, two combines); 2048 queries are all pairs; one query over one key
+    tile is a single unsplit launch."""
+    assert kvq.kvq_attention_launches(0, 12, 100) == 0
+    assert kvq.kvq_attention_launches(1, 1, 1) == 1
+    assert kvq.kvq_attention_launches(1560, 12, 93600) == 4
+    assert kvq.kvq_attention_launches(2048, 12, 93600) == 2
+
+
 def test_attention_rollout_shape_sampled(orc):
     """The rollout's attention at full size -- one frame of 1560 queries x 12 heads over a
     60-frame cache (93,600 keys) appended frame by frame with the mse rule -- checked on a

@@ -42,6 +42,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "kvq.h"
 #include "kvq_common.h"
@@ -114,7 +115,8 @@ struct AttnArgs {
     const uint8_t* vp;  // V cache
     const uint8_t* vs;
     const float* va;
-    int32_t n_q, heads, splits, key_tiles;
+    int32_t n_q, heads, key_tiles;
+    int32_t splits;            // partial results per row: gridDim.y, times 2 with DUAL
     int64_t n_kv;              // keys (tokens)
     int64_t tokens_per_chunk;  // keys per amax chunk
     float scale_log2;          // softmax scale * log2(e)
@@ -402,7 +404,33 @@ struct RawPiece {
     float amax;   // chunk amax of the key
 };
 
-__device__ __forceinline__ float global_scale(float amax) { return __fdiv_rn(amax, 2688.0f); }
+// gs = RN(amax / 2688). With MARK, without a division: Markstein's correction step (P.
+// Markstein, "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Dev. 34(1), 1990) with y = RN(1/2688): q = RN(amax y), r = amax - 2688 q
+// (exact as one fma), RN(q + r y). Compared with the IEEE quotient for every positive
+// finite fp32 amax, it differs only below 2^-119, where the quotient is subnormal; a
+// single CTA takes MARK when every chunk amax its keys use is in [2^-119, FLT_MAX] (the
+// IEEE division, with its rare slow path, in the producer loop cost 13 % of a single
+// CTA's time per key tile).
+constexpr float kMarkMinAmax = 0x1p-119f;
+constexpr int64_t kMarkScanMax = 4096;
+
+__device__ __forceinline__ bool markstein_amax(float amax)
+{
+    return amax >= kMarkMinAmax && amax <= 0x1.fffffep127f;
+}
+
+template <bool MARK>
+__device__ __forceinline__ float global_scale(float amax)
+{
+    if (MARK) {
+        constexpr float kInvDen = 0x1.861862p-12f;  // RN(1 / 2688)
+        const float q = __fmul_rn(amax, kInvDen);
+        const float r = __fmaf_rn(-q, 2688.0f, amax);
+        return __fmaf_rn(r, kInvDen, q);
+    }
+    return __fdiv_rn(amax, 2688.0f);
+}
 
 // Keys and chunk indices fit in 32 bits (a cache holds at most 2^36 elements, i.e. 2^29
 // rows of 128).
@@ -430,10 +458,11 @@ __device__ __forceinline__ uint32_t sw128r(int row, int kb, int chunk, int rows)
 // operand of Q K^T, V as the MN-major B operand of P V: the same bytes); a key past n_kv
 // gives zeros. With swap the two blocks are stored in the other order, so that threads
 // of neighbouring quarters hit different 16-byte bank groups of a shared-memory wavefront.
+template <bool MARK>
 __device__ __forceinline__ void store_piece(const RawPiece& r, bool valid, int row, int kb, int ch0, int rows,
                                             bool swap, uint32_t sT)
 {
-    const float gs = valid ? global_scale(r.amax) : 0.0f;
+    const float gs = valid ? global_scale<MARK>(r.amax) : 0.0f;
     const float SA = block_scale(r.sc, swap ? 1 : 0, gs), SB = block_scale(r.sc, swap ? 0 : 1, gs);
     const int s2 = swap ? 2 : 0;
     uint32_t y[4];
@@ -605,8 +634,9 @@ __device__ __forceinline__ float tile_row_exp(uint32_t tS, int valid, float scal
 // PAIR: the kernel runs as clusters of two CTAs (x even, x odd) that share every K/V
 // tile and issue cta_group::2 MMAs (M = 256: query tile slot g is rows 512 u + 256 g ..
 // + 255 of the pair, CTA `rank` holding the 128 from 512 u + 256 g + 128 rank); else one
-// CTA per unit of 256 query rows (slot g: rows 256 u + 128 g .. + 127).
-template <bool PAIR>
+// CTA per unit of 256 query rows (slot g: rows 256 u + 128 g .. + 127). DUAL: both slots
+// hold one query tile and split the CTA's key range (units of at most 128 rows).
+template <bool PAIR, bool DUAL>
 __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
 {
     using G = Geo<PAIR>;
@@ -618,23 +648,32 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = PAIR ? cluster_rank() : 0u;  // CTA 0 of a pair issues the MMAs
     const int unit = PAIR ? blockIdx.x >> 1 : blockIdx.x, split = blockIdx.y, h = blockIdx.z;
-    const int t_begin = static_cast<int>(static_cast<int64_t>(split) * a.key_tiles / a.splits);
-    const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * a.key_tiles / a.splits);
+    const int t_begin = static_cast<int>(static_cast<int64_t>(split) * a.key_tiles / gridDim.y);
+    const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * a.key_tiles / gridDim.y);
     const int n_tiles = t_end - t_begin;
     const int64_t u0 = static_cast<int64_t>(unit) * G::kRowsPerUnit;   // first row of the unit
     const int64_t q0 = u0 + rank * kBM;                                // this CTA's first row
     constexpr int kSlotRows = G::kCtas * kBM;                          // rows between slots
-    const int n_qt = a.n_q - u0 > kSlotRows ? 2 : 1;                   // slots holding rows
+    // dual: both slots hold query tile 0; slot 0 takes the first n_lead key tiles of the
+    // range, slot 1 the rest, and each writes its own partial result (2 split + slot)
+    constexpr bool dual = DUAL;
+    const int n_qt = dual || a.n_q - u0 > kSlotRows ? 2 : 1;         // slots in use
+    const int n_lead = dual ? (n_tiles + 1) >> 1 : n_tiles;          // slot 0's key tiles
+    auto slot_tiles = [&](int g) { return dual && g ? n_tiles - n_lead : n_lead; };
+    // the pipeline runs over stream tiles s: key tile t_begin + s, or with dual slot
+    // s % 2's tile s / 2; stream tile s lives in stage s % 2 with barrier phase (s / 2) % 2
+    auto key_tile = [&](int s) { return dual ? t_begin + ((s & 1) ? n_lead : 0) + (s >> 1) : t_begin + s; };
+    auto stream = [&](int g, int j) { return dual ? 2 * j + g : j; };
     const int64_t H = a.heads;
 
     const uint32_t base = (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) + 1023u) & ~1023u;
     const uint32_t bar0 = static_cast<uint32_t>(__cvta_generic_to_shared(&bars[0]));
     auto bar = [bar0](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-    // key tile j lives in K stage j % 2; its barriers' phase is j / 2
+    // stream tile s lives in K stage s % 2; its barriers' phase is s / 2
     auto sK = [base](int j) { return base + G::kOffK + static_cast<uint32_t>(j & 1) * G::kKBytes; };
     auto kfull = [&bar](int j) { return bar(kKFull0 + (j & 1)); };
     auto kempty = [&bar](int j) { return bar(kKEmpty0 + (j & 1)); };
-    // and so does value tile j in V stage j % 2
+    // and in V stage s % 2
     auto sV = [base](int j) { return base + G::kOffV + static_cast<uint32_t>(j & 1) * G::kVBytes; };
     auto vfull = [&bar](int j) { return bar(kVFull0 + (j & 1)); };
     auto vempty = [&bar](int j) { return bar(kVEmpty0 + (j & 1)); };
@@ -669,8 +708,8 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         mbar_init(bar(kMmaDone), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // both query tiles -> shared memory (rows past n_q are zero)
-    for (int i = tid; i < kQT * kBM * 16; i += kAttnThreads) {
+    // the query tiles -> shared memory (rows past n_q are zero; one tile with dual)
+    for (int i = tid; i < (dual ? 1 : kQT) * kBM * 16; i += kAttnThreads) {
         const int g = i >> 11, row = (i >> 4) & 127, kb = (i >> 3) & 1, ch = i & 7;
         const int64_t qrow = q0 + g * kSlotRows + row;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -678,9 +717,30 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
             v = ld_nc_v4(a.q + (qrow * H + h) * kD + kb * 64 + ch * 8);
         st_shared_v4(base + G::kOffQ + g * kTileBytes + sw128(row, kb, ch), v.x, v.y, v.z, v.w);
     }
+    // the correction step for the global scales if every chunk amax of the CTA's keys is
+    // in its exact range (a range over more than kMarkScanMax chunks takes the division).
+    // Only with DUAL, where the producers set the pace (each slot's chain has half the
+    // key tiles). A pair's producers, and those of a single CTA with two query tiles,
+    // wait for the softmax; there a second producer loop in the kernel measured 4-6 %
+    // slower overall.
+    constexpr bool producer_bound = !PAIR && DUAL;
+    int off_range = producer_bound ? 0 : 1;
+    if (producer_bound) {
+        const int64_t k_lo = static_cast<int64_t>(t_begin) * kBN;
+        const int64_t k_hi = min(static_cast<int64_t>(t_end) * kBN, a.n_kv);
+        if (k_hi > k_lo) {
+            const int64_t c0 = k_lo / a.tokens_per_chunk, c1 = (k_hi - 1) / a.tokens_per_chunk;
+            if (c1 - c0 >= kMarkScanMax)
+                off_range = 1;
+            else
+                for (int64_t c = c0 + tid; c <= c1; c += kAttnThreads)
+                    off_range |= static_cast<int>(!markstein_amax(__ldg(a.ka + c))) |
+                                 static_cast<int>(!markstein_amax(__ldg(a.va + c)));
+        }
+    }
     fence_async_smem();
     tc_before_sync();
-    __syncthreads();
+    const bool mark = __syncthreads_or(off_range) == 0;
     if (PAIR)
         cluster_sync();  // both CTAs' barriers initialized and TMEM allocated before any peer access
     tc_after_sync();
@@ -694,14 +754,15 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
             const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
             const uint32_t tS = tmem + g * 128 + lane_off, tO = tmem + 256 + g * 128 + lane_off;
             const uint32_t bS = bar(kSFull0 + g), bP = bar(kPFull0 + g), bO = bar(kODone0 + g);
+            const int my_tiles = slot_tiles(g);
             float m_run = -INFINITY, l_run = 0.0f;
             bool ok = true;
-            for (int j = 0; ok && j < n_tiles; ++j) {
+            for (int j = 0; ok && j < my_tiles; ++j) {
                 ok = warp_wait(bS, j & 1);
                 if (!ok)
                     break;
                 tc_after_sync();
-                const int64_t key0 = static_cast<int64_t>(t_begin + j) * kBN;
+                const int64_t key0 = static_cast<int64_t>(key_tile(stream(g, j))) * kBN;
                 const int valid = static_cast<int>(a.n_kv - key0 < kBN ? a.n_kv - key0 : kBN);
                 // the row max first; the reference moves (and O is rescaled) only when the
                 // max exceeds it by more than 2^8, which is rare after the first tiles
@@ -738,13 +799,23 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
                 if (lane == 0)
                     arrive_count<PAIR>(bP, 32);
             }
-            if (ok && n_tiles > 0) {
-                ok = warp_wait(bO, (n_tiles - 1) & 1);
+            if (ok && my_tiles == 0 && dual) {
+                // an empty key range (a one-tile range's slot 1): a partial of weight 0
+                const int64_t qrow = q0 + r;
+                const int64_t prow = (static_cast<int64_t>(2 * split + 1) * a.n_q + qrow) * H + h;
+                if (qrow < a.n_q) {
+                    for (int c = 0; c < kD; c += 4)
+                        st_v4(a.part_o + prow * kD + c, 0u, 0u, 0u, 0u);
+                    a.part_ml[prow] = make_float2(-INFINITY, 0.0f);
+                }
+            }
+            if (ok && my_tiles > 0) {
+                ok = warp_wait(bO, (my_tiles - 1) & 1);
                 if (ok) {
                     tc_after_sync();
-                    const int64_t qrow = q0 + g * kSlotRows + r;
+                    const int64_t qrow = q0 + (dual ? 0 : g * kSlotRows) + r;
                     const bool has_row = qrow < a.n_q;
-                    const int64_t prow = (static_cast<int64_t>(split) * a.n_q + qrow) * H + h;
+                    const int64_t prow = (static_cast<int64_t>(dual ? 2 * split + g : split) * a.n_q + qrow) * H + h;
                     const float inv_l = 1.0f / l_run;
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
@@ -779,44 +850,56 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
     } else if (warp == kMmaWarp) {
         // ---------------------------------------------------------------- MMA issue
         // (CTA 0 of a pair issues for both CTAs; CTA 1's MMA warp has nothing to do)
-        const uint32_t sQ0 = base + G::kOffQ, sQ1 = base + G::kOffQ + kTileBytes;
+        // Without dual both slots read each stream tile (one stage release per tile, after
+        // the last slot); with dual each stream tile belongs to one slot.
+        const uint32_t sQ0 = base + G::kOffQ, sQ1 = dual ? sQ0 : base + G::kOffQ + kTileBytes;
         bool ok = true;
-        const int tiles = rank == 0 ? n_tiles : 0;
-        if (tiles > 0) {
-            ok = warp_wait(kfull(0), 0);
-            if (ok) {
-                tc_after_sync();
-                mma_qk<PAIR>(tmem, sQ0, sK(0));
-                commit<PAIR>(bar(kSFull0));
-                if (n_qt == 2) {
-                    mma_qk<PAIR>(tmem + 128, sQ1, sK(0));
-                    commit<PAIR>(bar(kSFull1));
+        const int steps = rank == 0 ? n_lead : 0;
+        if (steps > 0) {
+            // S_g(0) for each slot: stream tile 0 for both, or with dual tiles 0 and 1
+            for (int g = 0; ok && g < n_qt; ++g) {
+                if (slot_tiles(g) == 0)
+                    break;
+                const int s = stream(g, 0);
+                if (g == 0 || dual) {
+                    ok = warp_wait(kfull(s), 0);
+                    if (!ok)
+                        break;
+                    tc_after_sync();
                 }
-                commit<PAIR>(kempty(0));
+                mma_qk<PAIR>(tmem + g * 128, g == 0 ? sQ0 : sQ1, sK(s));
+                commit<PAIR>(bar(kSFull0 + g));
+                if (dual || g == n_qt - 1)
+                    commit<PAIR>(kempty(s));
             }
         }
-        for (int j = 0; ok && j < tiles; ++j) {
+        for (int j = 0; ok && j < steps; ++j) {
             for (int g = 0; g < n_qt; ++g) {
-                // O_g += P_g V(j), then S_g(j+1) = Q_g K(j+1)^T
-                ok = warp_wait(bar(kPFull0 + g), j & 1) && (g > 0 || warp_wait(vfull(j), (j >> 1) & 1));
+                // O_g += P_g V(s), then S_g(j+1) = Q_g K(s')^T for the slot's next tile s'
+                const int gt = slot_tiles(g), s = stream(g, j);
+                if (j >= gt)
+                    break;
+                ok = warp_wait(bar(kPFull0 + g), j & 1) &&
+                     ((g > 0 && !dual) || warp_wait(vfull(s), (s >> 1) & 1));
                 if (!ok)
                     break;
                 tc_after_sync();
-                mma_pv<PAIR>(tmem + 256 + g * 128, tmem + g * 128, sV(j), j > 0);
+                mma_pv<PAIR>(tmem + 256 + g * 128, tmem + g * 128, sV(s), j > 0);
                 commit<PAIR>(bar(kODone0 + g));
-                if (g == n_qt - 1)
-                    commit<PAIR>(vempty(j));
-                if (j + 1 < tiles) {
-                    if (g == 0) {
-                        ok = warp_wait(kfull(j + 1), ((j + 1) >> 1) & 1);
+                if (dual || g == n_qt - 1)
+                    commit<PAIR>(vempty(s));
+                if (j + 1 < gt) {
+                    const int s2 = stream(g, j + 1);
+                    if (g == 0 || dual) {
+                        ok = warp_wait(kfull(s2), (s2 >> 1) & 1);
                         if (!ok)
                             break;
                         tc_after_sync();
                     }
-                    mma_qk<PAIR>(tmem + g * 128, g == 0 ? sQ0 : sQ1, sK(j + 1));
+                    mma_qk<PAIR>(tmem + g * 128, g == 0 ? sQ0 : sQ1, sK(s2));
                     commit<PAIR>(bar(kSFull0 + g));
-                    if (g == n_qt - 1)
-                        commit<PAIR>(kempty(j + 1));
+                    if (dual || g == n_qt - 1)
+                        commit<PAIR>(kempty(s2));
                 }
             }
         }
@@ -838,70 +921,109 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         // (p + 256 i) / 4 of this CTA's key rows, quarter p % 4; V key row (p + 256 i) /
         // kVQuarters, quarter p % kVQuarters of this CTA's dims. A warp's arrivals are one
         // arrive of 32 (on CTA 0's barrier with PAIR).
-        const int p = tid - kSoftmaxThreads;
-        auto key0_of = [&](int j) { return static_cast<int64_t>(t_begin + j) * kBN; };
-        const int k_q = p & 3, v_q = p % G::kVQuarters;
-        auto k_row = [&](int i) { return (p + kProducerThreads * i) >> 2; };
-        auto v_row = [&](int i) { return (p + kProducerThreads * i) / G::kVQuarters; };
-        auto k_key = [&](int j, int i) { return key0_of(j) + rank * (kBN - G::kKRows) + k_row(i); };
-        auto v_key = [&](int j, int i) { return key0_of(j) + v_row(i); };
-        RawPiece rk[G::kKPieces], rv[G::kVPieces];
-        auto load_k = [&](int j) {
-#pragma unroll
-            for (int i = 0; i < G::kKPieces; ++i)
-                load_piece(a.kp, a.ks, a.ka, a, h, k_key(j, i), k_q, rk[i]);
-        };
-        auto load_v = [&](int j) {
-#pragma unroll
-            for (int i = 0; i < G::kVPieces; ++i)
-                load_piece(a.vp, a.vs, a.va, a, h, v_key(j, i), v_q + static_cast<int>(rank) * G::kVQuarters, rv[i]);
-        };
-        auto put_k = [&](int j) {
-#pragma unroll
-            for (int i = 0; i < G::kKPieces; ++i)
-                store_piece(rk[i], k_key(j, i) < a.n_kv, k_row(i), k_q >> 1, (k_q & 1) * 4, G::kKRows, (k_q & 2) != 0,
-                            sK(j));
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                arrive_count<PAIR>(kfull(j), 32);
-        };
-        auto put_v = [&](int j) {
-#pragma unroll
-            for (int i = 0; i < G::kVPieces; ++i)
-                store_piece(rv[i], v_key(j, i) < a.n_kv, v_row(i), v_q >> 1, (v_q & 1) * 4, kBN, (v_q & 2) != 0,
-                            sV(j));
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                arrive_count<PAIR>(vfull(j), 32);
-        };
-        bool ok = true;
-        if (n_tiles > 0) {
-            load_k(0);
-            load_v(0);
-            put_k(0);
-            if (n_tiles > 1)
-                load_k(1);
-        }
-        for (int j = 0; j < n_tiles; ++j) {
-            if (j + 1 < n_tiles) {
-                // stage (j+1) % 2 was last read by the S MMAs of key tile j - 1
-                if (j > 0 && !(ok = wait_phase(kempty(j + 1), (((j + 1) >> 1) - 1) & 1)))
-                    break;
-                put_k(j + 1);
-                if (j + 2 < n_tiles)
-                    load_k(j + 2);
+        // the producer loop, with the global scale by the correction step (MARK) or by
+        // IEEE division; the choice is uniform over the CTA
+        auto produce = [&](auto mark_tag) {
+            constexpr bool MARK = decltype(mark_tag)::value;
+            const int p = tid - kSoftmaxThreads;
+            auto key0_of = [&](int s) { return static_cast<int64_t>(key_tile(s)) * kBN; };
+            const int k_q = p & 3, v_q = p % G::kVQuarters;
+            auto k_row = [&](int i) { return (p + kProducerThreads * i) >> 2; };
+            auto v_row = [&](int i) { return (p + kProducerThreads * i) / G::kVQuarters; };
+            auto k_key = [&](int j, int i) { return key0_of(j) + rank * (kBN - G::kKRows) + k_row(i); };
+            auto v_key = [&](int j, int i) { return key0_of(j) + v_row(i); };
+            RawPiece rk[G::kKPieces], rv[G::kVPieces];
+            auto load_k = [&](int j) {
+    #pragma unroll
+                for (int i = 0; i < G::kKPieces; ++i)
+                    load_piece(a.kp, a.ks, a.ka, a, h, k_key(j, i), k_q, rk[i]);
+            };
+            auto load_v = [&](int j) {
+    #pragma unroll
+                for (int i = 0; i < G::kVPieces; ++i)
+                    load_piece(a.vp, a.vs, a.va, a, h, v_key(j, i), v_q + static_cast<int>(rank) * G::kVQuarters, rv[i]);
+            };
+            auto put_k = [&](int j) {
+    #pragma unroll
+                for (int i = 0; i < G::kKPieces; ++i)
+                    store_piece<MARK>(rk[i], k_key(j, i) < a.n_kv, k_row(i), k_q >> 1, (k_q & 1) * 4, G::kKRows, (k_q & 2) != 0,
+                                sK(j));
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    arrive_count<PAIR>(kfull(j), 32);
+            };
+            auto put_v = [&](int j) {
+    #pragma unroll
+                for (int i = 0; i < G::kVPieces; ++i)
+                    store_piece<MARK>(rv[i], v_key(j, i) < a.n_kv, v_row(i), v_q >> 1, (v_q & 1) * 4, kBN, (v_q & 2) != 0,
+                                sV(j));
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    arrive_count<PAIR>(vfull(j), 32);
+            };
+            bool ok = true;
+            if (dual) {
+                // the MMA warp takes S(0), S(1), then P V(s) and S(s + 2) for each stream tile
+                // s; stage s % 2 of K is freed by S(s), of V by P V(s)
+                load_k(0);
+                load_v(0);
+                put_k(0);
+                if (n_tiles > 1) {
+                    load_k(1);
+                    put_k(1);
+                    if (n_tiles > 2)
+                        load_k(2);
+                }
+                for (int s = 0; s < n_tiles; ++s) {
+                    if (s > 1 && !(ok = wait_phase(vempty(s), ((s >> 1) - 1) & 1)))
+                        break;
+                    put_v(s);
+                    if (s + 1 < n_tiles)
+                        load_v(s + 1);
+                    if (s + 2 < n_tiles) {
+                        if (!(ok = wait_phase(kempty(s + 2), (s >> 1) & 1)))
+                            break;
+                        put_k(s + 2);
+                        if (s + 3 < n_tiles)
+                            load_k(s + 3);
+                    }
+                }
+                if (!ok && lane == 0)
+                    atomicExch(a.status, 1);
+            } else {
+            if (n_tiles > 0) {
+                load_k(0);
+                load_v(0);
+                put_k(0);
+                if (n_tiles > 1)
+                    load_k(1);
             }
-            // stage j % 2 was last read by the P V MMAs of value tile j - 2
-            if (j > 1 && !(ok = wait_phase(vempty(j), ((j >> 1) - 1) & 1)))
-                break;
-            put_v(j);
-            if (j + 1 < n_tiles)
-                load_v(j + 1);
-        }
-        if (!ok && lane == 0)
-            atomicExch(a.status, 1);
+            for (int j = 0; j < n_tiles; ++j) {
+                if (j + 1 < n_tiles) {
+                    // stage (j+1) % 2 was last read by the S MMAs of key tile j - 1
+                    if (j > 0 && !(ok = wait_phase(kempty(j + 1), (((j + 1) >> 1) - 1) & 1)))
+                        break;
+                    put_k(j + 1);
+                    if (j + 2 < n_tiles)
+                        load_k(j + 2);
+                }
+                // stage j % 2 was last read by the P V MMAs of value tile j - 2
+                if (j > 1 && !(ok = wait_phase(vempty(j), ((j >> 1) - 1) & 1)))
+                    break;
+                put_v(j);
+                if (j + 1 < n_tiles)
+                    load_v(j + 1);
+            }
+            if (!ok && lane == 0)
+                atomicExch(a.status, 1);
+            }
+        };
+        if (producer_bound && mark)
+            produce(std::integral_constant<bool, producer_bound>{});
+        else
+            produce(std::false_type{});
     }
     tc_before_sync();
     __syncthreads();
@@ -990,17 +1112,20 @@ bool cluster_launch_supported()
 // (CTA pairs or single CTAs) with its key splits, workspace region and combine. A pair's
 // steady state takes about 15/16 of the time per query row of a single CTA (its M = 256
 // MMAs occupy each SM 76 cycles against 95 for M = 128; measured 7 % faster at 1024 and
-// 2048 queries), but its unit is 512 rows against 256. In units of a single CTA's time
-// per key tile, all single costs 16 ceil(n / 256), all pairs 30 ceil(n / 512), and pairs
-// over the whole 512-row blocks with single CTAs for the rest 30 floor(n / 512) +
-// 16 ceil((n mod 512) / 256); the cheapest wins (ties to fewer launches). 1560 queries
-// take three pairs for 1536 rows and one single CTA for the last 24.
+// 2048 queries), but its unit is 512 rows against 256. A single CTA whose rows fit one
+// query tile (at most 128) runs dual: its two slots split the CTA's key range, which
+// halves the serial chain of key tiles (a one-tile step costs about as much as a two-tile
+// step). In units of a single CTA's time per key tile, a single unit costs 16 (8 when
+// dual), a pair unit 30; the plan takes the cheapest of all single CTAs, all pairs, and
+// pairs over the whole 512-row blocks with single CTAs for the rest (ties to fewer
+// launches). 1560 queries take three pairs for 1536 rows and one dual CTA for the last 24.
 struct AttnPart {
-    bool pair;
+    bool pair, dual;
     int32_t row0, rows;  // query rows [row0, row0 + rows)
     int64_t units;
-    int splits;
+    int splits;          // key ranges (gridDim.y); partial results per row: splits << dual
     uint64_t ws_offset;  // of its partials in the workspace
+    int partials() const { return splits << (dual ? 1 : 0); }
 };
 
 struct AttnPlan {
@@ -1016,29 +1141,37 @@ void finish_plan(AttnPlan& pl, int32_t heads)
     uint64_t off = 0;
     for (int i = 0; i < pl.n_parts; ++i) {
         pl.part[i].ws_offset = off;
-        off += (partial_bytes(pl.part[i].splits, pl.part[i].rows, heads) + kWsAlign - 1) / kWsAlign * kWsAlign;
+        off += (partial_bytes(pl.part[i].partials(), pl.part[i].rows, heads) + kWsAlign - 1) / kWsAlign * kWsAlign;
     }
     pl.ws_bytes = off;
 }
 
+int64_t single_cost(int32_t rows)
+{
+    return rows <= kBM ? 8 : 16 * ((rows + Geo<false>::kRowsPerUnit - 1) / Geo<false>::kRowsPerUnit);
+}
+
 AttnPlan plan_attention(int32_t n_q, int32_t heads, int64_t key_tiles)
 {
-    constexpr int32_t kSingleRows = Geo<false>::kRowsPerUnit, kPairRows = Geo<true>::kRowsPerUnit;
-    const int64_t cost_single = 16 * ((n_q + kSingleRows - 1) / kSingleRows);
+    constexpr int32_t kPairRows = Geo<true>::kRowsPerUnit;
+    const int64_t cost_single = single_cost(n_q);
     const int64_t cost_pair = 30 * ((n_q + kPairRows - 1) / kPairRows);
     const int32_t full_rows = n_q / kPairRows * kPairRows, rest = n_q - full_rows;
-    const int64_t cost_mixed = 30 * (full_rows / kPairRows) + 16 * ((rest + kSingleRows - 1) / kSingleRows);
+    const int64_t cost_mixed = 30 * (full_rows / kPairRows) + (rest > 0 ? single_cost(rest) : 0);
     const bool pairs_ok = cluster_launch_supported();
+    const int sms = sm_count();
     AttnPlan pl{};
     auto part = [&](bool pair, int32_t row0, int32_t rows) {
-        const int32_t unit_rows = pair ? kPairRows : kSingleRows;
+        const int32_t unit_rows = pair ? kPairRows : Geo<false>::kRowsPerUnit;
         AttnPart pt{};
         pt.pair = pair;
         pt.row0 = row0;
         pt.rows = rows;
         pt.units = (rows + unit_rows - 1) / unit_rows;
-        const int sms = sm_count();
-        pt.splits = choose_splits(pt.units * heads, static_cast<int>(key_tiles), pair ? sms / 2 : sms);
+        // dual needs at least two key tiles per CTA: the split is chosen over half the tiles
+        pt.dual = !pair && rows <= kBM && key_tiles >= 2;
+        const int kt = static_cast<int>(pt.dual ? key_tiles / 2 : key_tiles);
+        pt.splits = choose_splits(pt.units * heads, kt, pair ? sms / 2 : sms);
         return pt;
     };
     if (!pairs_ok || (cost_single <= cost_pair && cost_single <= cost_mixed)) {
@@ -1060,17 +1193,18 @@ AttnPlan plan_attention(int32_t n_q, int32_t heads, int64_t key_tiles)
 // CTA's launch allocation, so the split balances only if the kernel is launched with
 // exactly kLaunchRegs registers per thread: refuse to launch otherwise, since an
 // unbalanced split would wait for registers forever), set the shared-memory size, launch.
-template <bool PAIR>
+template <bool PAIR, bool DUAL>
 kvq_status launch_attention(const AttnArgs& a, int64_t units, int splits, int heads, cudaStream_t stream)
 {
     cudaFuncAttributes fa{};
-    cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel<PAIR>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, attention_kernel<PAIR, DUAL>);
     if (e != cudaSuccess)
         return launched(e, "kvq_attention");
     if (fa.numRegs != kLaunchRegs)
         return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: kernel built with %d registers per thread, its register split needs %d",
                     fa.numRegs, kLaunchRegs);
-    e = cudaFuncSetAttribute(attention_kernel<PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<PAIR>::kSmemBytes);
+    e = cudaFuncSetAttribute(attention_kernel<PAIR, DUAL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Geo<PAIR>::kSmemBytes);
     if (e != cudaSuccess)
         return launched(e, "kvq_attention");
     cudaLaunchAttribute attr[2];
@@ -1088,7 +1222,7 @@ kvq_status launch_attention(const AttnArgs& a, int64_t units, int splits, int he
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
-    return launched(cudaLaunchKernelEx(&cfg, attention_kernel<PAIR>, a), "kvq_attention");
+    return launched(cudaLaunchKernelEx(&cfg, attention_kernel<PAIR, DUAL>, a), "kvq_attention");
 }
 
 }  // namespace
@@ -1124,7 +1258,7 @@ kvq_status kvq_attention_launches(int32_t n_queries, int32_t heads, int64_t n_ke
         return fail(KVQ_ERR_INVALID_ARG, "kvq_attention_launches: too many keys");
     const AttnPlan plan = plan_attention(n_queries, heads, key_tiles);
     for (int i = 0; i < plan.n_parts; ++i)
-        *launches += plan.part[i].splits > 1 ? 2 : 1;
+        *launches += plan.part[i].partials() > 1 ? 2 : 1;
     return ok();
 }
 
@@ -1168,13 +1302,18 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
         return fail(KVQ_ERR_INVALID_ARG, "kvq_attention: too many keys");
     if (static_cast<int64_t>(n_queries) * heads / (kCombineThreads / 32) >= INT32_MAX)
         return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention: n_queries * heads too large");
-    // a workspace smaller than the plan's takes fewer key splits, the larger split first
+    // a workspace smaller than the plan's takes fewer key splits (the part with the most
+    // partials first), and in the end no dual
     AttnPlan plan = plan_attention(n_queries, heads, key_tiles);
     while (plan.ws_bytes > workspace_bytes) {
-        AttnPart& big = plan.n_parts == 2 && plan.part[1].splits > plan.part[0].splits ? plan.part[1] : plan.part[0];
-        if (big.splits <= 1)
+        AttnPart& big =
+            plan.n_parts == 2 && plan.part[1].partials() > plan.part[0].partials() ? plan.part[1] : plan.part[0];
+        if (big.splits > 1)
+            --big.splits;
+        else if (big.dual)
+            big.dual = false;
+        else
             break;
-        --big.splits;
         finish_plan(plan, heads);
     }
     if (plan.ws_bytes > 0 && (workspace == nullptr || !aligned(workspace, 16)))
@@ -1188,9 +1327,10 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
         AttnArgs a;
         a.q = static_cast<const uint16_t*>(q) + row_off;
         a.o = static_cast<uint16_t*>(out) + row_off;
-        a.part_o = pt.splits > 1 ? part_ws : nullptr;
-        a.part_ml = pt.splits > 1 ? reinterpret_cast<float2*>(part_ws + static_cast<uint64_t>(pt.splits) * pt.rows * heads * kD)
-                                  : nullptr;
+        const int partials = pt.partials();
+        a.part_o = partials > 1 ? part_ws : nullptr;
+        a.part_ml = partials > 1 ? reinterpret_cast<float2*>(part_ws + static_cast<uint64_t>(partials) * pt.rows * heads * kD)
+                                 : nullptr;
         a.kp = k_cache->packed;
         a.ks = k_cache->scales;
         a.ka = k_cache->amax;
@@ -1199,18 +1339,20 @@ kvq_status kvq_attention(const void* q, int32_t n_queries, int32_t heads, const 
         a.va = v_cache->amax;
         a.n_q = pt.rows;
         a.heads = heads;
-        a.splits = pt.splits;
+        a.splits = partials;
         a.key_tiles = static_cast<int32_t>(key_tiles);
         a.n_kv = n_keys;
         a.tokens_per_chunk = k_cache->rows_per_chunk / heads;
         a.scale_log2 = softmax_scale * 1.4426950408889634f;
         a.status = status;
 
-        kvq_status st = pt.pair ? launch_attention<true>(a, pt.units, pt.splits, heads, s)
-                                : launch_attention<false>(a, pt.units, pt.splits, heads, s);
+        // (the plan takes dual only for single CTAs)
+        kvq_status st = pt.pair   ? launch_attention<true, false>(a, pt.units, pt.splits, heads, s)
+                        : pt.dual ? launch_attention<false, true>(a, pt.units, pt.splits, heads, s)
+                                  : launch_attention<false, false>(a, pt.units, pt.splits, heads, s);
         if (st != KVQ_OK)
             return st;
-        if (pt.splits == 1)
+        if (partials == 1)
             continue;
         const int64_t rows = static_cast<int64_t>(pt.rows) * heads;
         const int64_t rows_per_cta = kCombineThreads / 32;

@@ -94,6 +94,9 @@ def _workspace(split):
     # CTA pairs (cta_group::2) take these: 2 x 15/16 x ceil(n_q / 512) < ceil(n_q / 256)
     (400, 2, 300, 100, "mse"),       # one pair; CTA 1's second slot holds 16 rows
     (1024, 1, 385, 64, "static_6"),  # two full pairs, a partial last key tile
+    # at most 128 rows: the CTA's two slots split its key range (dual); with two key
+    # ranges of 2 and 3 tiles, the second range's slots take 2 and 1, the last ragged
+    (100, 2, 5 * 128 - 7, 100, "static_4"),
 ])
 def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rule, split):
     caches, ocs = _filled_caches(orc, heads, n_keys, tokens_per_chunk, rule, 100)
@@ -143,6 +146,31 @@ def test_workspace_size_and_split_agree():
     assert kvq.kvq_attention_workspace_bytes(1, 1, 1) == 0
     b = kvq.kvq_attention_workspace_bytes(1560, 12, 93600)
     assert b >= 2 * 1560 * 12 * (128 * 4 + 8) and b % 256 == 0
+
+
+@pytest.mark.parametrize("log2_scale", [-133, -125, -121, -119, -118, -100, -40, 0, 40, 100, 120])
+def test_attention_dequantizes_like_the_cache_reader(log2_scale):
+    """The K/V tiles the attention kernel dequantizes on chip are the bf16 values
+    kvq_dequantize_cache writes, bit for bit, whatever the chunk amax: with one key and
+    zero queries, softmax gives p = 1 and the output is that key's V row exactly. The
+    scales 2^-133 .. 2^120 cover amax whose global scale amax / 2688 is subnormal (the
+    kernel then divides) and the normal range (it uses a correction step). At 2^-133
+    every value dequantizes to a signed zero."""
+    heads, n_q = 4, 3
+    x = (inputs.normal((1, heads, D), 1000 + log2_scale, "cuda").double() * 2.0 ** log2_scale).to(torch.bfloat16)
+    caches = [kvq.KVCache(heads, heads, D) for _ in range(2)]
+    for c in caches:
+        kvq.kvq_append(c, 0, x, "mse")
+    q = torch.zeros((n_q, heads, D), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], 1, status=status)
+    v = kvq.kvq_dequantize_cache(caches[1], 0, heads).view(1, heads, D)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    # compared as values: equal bf16 values have equal bits, except -0, which the sum
+    # P V turns into +0
+    want = v.expand(n_q, heads, D).float()
+    assert torch.equal(out.float(), want)
 
 
 def test_attention_launch_count():

@@ -1113,11 +1113,11 @@ bool cluster_launch_supported()
 // steady state takes about 15/16 of the time per query row of a single CTA (its M = 256
 // MMAs occupy each SM 76 cycles against 95 for M = 128; measured 7 % faster at 1024 and
 // 2048 queries), but its unit is 512 rows against 256. A single CTA whose rows fit one
-// query tile (at most 128) runs dual: its two slots split the CTA's key range, which
-// halves the serial chain of key tiles (a one-tile step costs about as much as a two-tile
-// step). In units of a single CTA's time per key tile, a single unit costs 16 (8 when
-// dual), a pair unit 30; the plan takes the cheapest of all single CTAs, all pairs, and
-// pairs over the whole 512-row blocks with single CTAs for the rest (ties to fewer
+// query tile (at most 128) runs dual: its two slots split the CTA's key range, and its
+// producers, which then set the pace, skip the division (measured 0.74 of a two-tile
+// unit's time). In units of a single CTA's time per key tile, a single unit costs 16 (12
+// when dual), a pair unit 30; the plan takes the cheapest of all single CTAs, all pairs,
+// and pairs over the whole 512-row blocks with single CTAs for the rest (ties to fewer
 // launches). 1560 queries take three pairs for 1536 rows and one dual CTA for the last 24.
 struct AttnPart {
     bool pair, dual;
@@ -1148,7 +1148,7 @@ void finish_plan(AttnPlan& pl, int32_t heads)
 
 int64_t single_cost(int32_t rows)
 {
-    return rows <= kBM ? 8 : 16 * ((rows + Geo<false>::kRowsPerUnit - 1) / Geo<false>::kRowsPerUnit);
+    return rows <= kBM ? 12 : 16 * ((rows + Geo<false>::kRowsPerUnit - 1) / Geo<false>::kRowsPerUnit);
 }
 
 AttnPlan plan_attention(int32_t n_q, int32_t heads, int64_t key_tiles)

@@ -12,7 +12,12 @@
 // tiles (128 keys each). When the keys are split over several units, each leaves a
 // partial result (unnormalized O, reference max m and sum l per row) in the caller's
 // workspace and combine_kernel merges them; the split count is chosen so the units fill
-// the SMs in whole waves.
+// the SMs in whole waves. Three instantiations: single CTAs; CTA pairs (PAIR: a cluster
+// of two issuing cta_group::2 MMAs with M = 256, each CTA holding its own 2 x 128 rows
+// and dequantizing half of every K and V tile); and single CTAs whose two slots share
+// one query tile and split the key range (DUAL, for units of at most 128 rows). The
+// host splits the query rows into at most two launches (pairs over whole 512-row
+// blocks, single or dual CTAs for the rest) by a cost model measured on this part.
 //
 // Roles inside the CTA (544 threads, 17 warps):
 //   warps 0-3, 4-7  softmax of query tile 0 / 1: thread t owns row t (TMEM lane t). Per

@@ -20,7 +20,8 @@
 // blocks, single or dual CTAs for the rest) by a cost model measured on this part.
 //
 // Roles inside the CTA (544 threads, 17 warps):
-//   warps 0-3, 4-7  softmax of query tile 0 / 1: thread t owns row t (TMEM lane t). Per
+//   warps 0-3, 4-7  softmax of query tile 0 / 1 (with DUAL both take tile 0, each over
+//                   its half of the key range): thread t owns row t (TMEM lane t). Per
 //                   key tile: the row max of S first, then p = 2^(s - m) written as bf16
 //                   into TMEM over the S columns already read. Warp 0 allocates and frees
 //                   the TMEM.

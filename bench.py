@@ -832,20 +832,27 @@ class Attention:
 
     def oracle_sample(self, orc, inputs, budget_s):
         """Layer 0: the oracle appends the cache (untimed), then dequantizes K and V and
-        computes a few query rows' attention in fp64 (timed); the bytes are the layer's
-        algorithmic bytes scaled by the share of query rows done."""
+        computes query rows' attention in fp64 (timed), doubling the rows per batch until
+        the time budget is spent; the bytes are the layer's algorithmic bytes scaled by
+        the share of query rows done."""
         caches = [orc.Cache(self.frames * self.rpc, self.rpc, self.D) for _ in range(2)]
         for f in range(self.frames):
             for t in range(2):
                 caches[t].append(f * self.rpc, inputs.bits(inputs.rollout_chunk(f, t, heads=self.heads,
                                                                                 tokens=self.tokens)), self.rule)
         qb = inputs.bits(inputs.queries(0, heads=self.heads, tokens=self.tokens)).reshape(self.tokens, -1)
-        m = 4
         t0 = time.perf_counter()
         kb, vb = caches[0].dequantize(0, self.n_keys * self.heads), caches[1].dequantize(0, self.n_keys * self.heads)
-        orc.attention(qb[:m].reshape(-1), kb, vb, m, self.n_keys, self.heads, self.D, self.D ** -0.5)
+        rows, m = 0, 4
+        while rows < self.tokens:
+            m = min(m, self.tokens - rows)
+            orc.attention(qb[rows:rows + m].reshape(-1), kb, vb, m, self.n_keys, self.heads, self.D, self.D ** -0.5)
+            rows += m
+            if time.perf_counter() - t0 >= budget_s:
+                break
+            m *= 2
         dt = time.perf_counter() - t0
-        return self.bytes_layer * m / self.tokens, dt, f"layer 0, {m} of {self.tokens} query rows"
+        return self.bytes_layer * rows / self.tokens, dt, f"layer 0, {rows} of {self.tokens} query rows"
 
 
 WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention, Recent, Layout)}

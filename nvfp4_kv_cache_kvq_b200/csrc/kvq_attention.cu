@@ -1152,23 +1152,23 @@ void finish_plan(AttnPlan& pl, int32_t heads)
     pl.ws_bytes = off;
 }
 
-int64_t single_cost(int32_t rows)
+int64_t single_cost(int64_t rows)
 {
     return rows <= kBM ? 12 : 16 * ((rows + Geo<false>::kRowsPerUnit - 1) / Geo<false>::kRowsPerUnit);
 }
 
 AttnPlan plan_attention(int32_t n_q, int32_t heads, int64_t key_tiles)
 {
-    constexpr int32_t kPairRows = Geo<true>::kRowsPerUnit;
+    constexpr int64_t kPairRows = Geo<true>::kRowsPerUnit;
     const int64_t cost_single = single_cost(n_q);
-    const int64_t cost_pair = 30 * ((n_q + kPairRows - 1) / kPairRows);
-    const int32_t full_rows = n_q / kPairRows * kPairRows, rest = n_q - full_rows;
+    const int64_t cost_pair = 30 * ((n_q + kPairRows - 1) / kPairRows);  // 64-bit: n_q may be near 2^31
+    const int32_t full_rows = static_cast<int32_t>(n_q / kPairRows * kPairRows), rest = n_q - full_rows;
     const int64_t cost_mixed = 30 * (full_rows / kPairRows) + (rest > 0 ? single_cost(rest) : 0);
     const bool pairs_ok = cluster_launch_supported();
     const int sms = sm_count();
     AttnPlan pl{};
     auto part = [&](bool pair, int32_t row0, int32_t rows) {
-        const int32_t unit_rows = pair ? kPairRows : Geo<false>::kRowsPerUnit;
+        const int64_t unit_rows = pair ? kPairRows : Geo<false>::kRowsPerUnit;
         AttnPart pt{};
         pt.pair = pair;
         pt.row0 = row0;

@@ -35,6 +35,9 @@
  *     the even code, saturating at 6, sign kept, so negative values that round to
  *     zero give code 0x8). When 1/S is infinite (S == 0) every product is x * 0.
  *   - rule mse keeps R = 4 only when its squared error is strictly smaller than R = 6's.
+ *     The pages fix no evaluation order for that error; the order used (block_sq_error)
+ *     is pinned by hand-worked near-tie blocks and an exact-rational restatement of
+ *     the quantizer in the tests.
  *   - the even-indexed element of a pair goes in the low nibble.
  *   - dequant: y = bf16_rne(e2m1_value(q) * S), the product rounded to fp32 first.
  *

@@ -227,6 +227,8 @@ class Rollout:
         self.layers, self.heads, self.tokens, self.frames, self.D = 30, 12, 1560, 60, 128
         if args.small:
             self.layers, self.heads, self.tokens, self.frames = 2, 2, 120, 6
+        if args.frames:  # fewer frames of the same shape (profiling)
+            self.frames = args.frames
         self.rule = args.rule or "mse"
         self.rank = rank
         self.rpc = self.tokens * self.heads
@@ -261,7 +263,7 @@ class Rollout:
 
             def app(f=f, xs=xs):
                 kvq.kvq_append_batch(self.caches, [f * self.rpc] * T, xs, self.rule)
-            segs.append(Segment("append", app, 3 * math.ceil(T / kvq.MAX_BATCH),
+            segs.append(Segment("append", app, kvq.kvq_quantize_launches(T, self.chunk_elems, self.D),
                                 T * self.chunk_elems * (B_AMAX + B_QUANT), h2d=(self.x[f],)))
             rows = (f + 1) * self.rpc
 
@@ -370,7 +372,8 @@ class Layer:
 
         def d():
             kvq.kvq_dequantize_batch(self.p[:m], self.s[:m], self.a[:m], self.D, ys=self.y[:m])
-        return [Segment("quantize", q, 3, m * self.n * (B_AMAX + B_QUANT), h2d=tuple(self.x)),
+        return [Segment("quantize", q, kvq.kvq_quantize_launches(m, self.n, self.D), m * self.n * (B_AMAX + B_QUANT),
+                        h2d=tuple(self.x)),
                 Segment("dequant", d, 1, m * self.n * B_DEQUANT)]
 
     def d2h(self):
@@ -433,7 +436,7 @@ class Cache:
             for l in range(self.layers):
                 kvq.kvq_dequantize_batch([self.p[2 * l], self.p[2 * l + 1]], [self.s[2 * l], self.s[2 * l + 1]],
                                          [self.a[2 * l], self.a[2 * l + 1]], self.D, ys=[self.y[0], self.y[1]])
-        return [Segment("quantize", q, 3 * math.ceil(T / self.kvq.MAX_BATCH), T * self.n * (B_AMAX + B_QUANT),
+        return [Segment("quantize", q, kvq.kvq_quantize_launches(T, self.n, self.D), T * self.n * (B_AMAX + B_QUANT),
                         h2d=(self.x,)),
                 Segment("dequant", d, self.layers, T * self.n * B_DEQUANT)]
 
@@ -544,7 +547,8 @@ class RoundTrip(Sweep):
         def rt():
             kvq.kvq_quantize_dequantize(self.x[0], self.D, self.rule, amax_out=self.a[0], packed=self.p[0],
                                         scales=self.s[0], y=self.y[0])
-        return [Segment("roundtrip", rt, 3, self.n * (B_AMAX + B_QUANT + 2.0), h2d=(self.x[0],))]
+        return [Segment("roundtrip", rt, kvq.kvq_quantize_launches(1, self.n, self.D), self.n * (B_AMAX + B_QUANT + 2.0),
+                        h2d=(self.x[0],))]
 
     def d2h(self):
         return [self.p[0], self.s[0], self.a[0], self.y[0]]
@@ -1021,6 +1025,7 @@ def main():
     ap.add_argument("--bits", type=int, choices=(2, 4), default=4, help="bits of the rtn workload")
     ap.add_argument("--small", action="store_true", help="a reduced shape of the workload (for tests)")
     ap.add_argument("--layers", type=int, default=None, help="layers of the attention workload (profiling)")
+    ap.add_argument("--frames", type=int, default=None, help="frames of the rollout workload (profiling)")
     ap.add_argument("--no-graphs", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -34,8 +34,9 @@
  * Conventions for every call:
  *   - Pointers named "device" are CUDA device (or managed) memory that the caller
  *     allocates, owns and frees. The library never allocates or frees memory and keeps
- *     no state between calls, with one stated exception: kvq_attention_noalloc's
- *     built-in scratch array (see there). Host pointers are read before the call returns.
+ *     no state between calls, with two stated exceptions: kvq_attention_noalloc's
+ *     built-in scratch array (see there) and the per-device error word that
+ *     kvq_device_status reads. Host pointers are read before the call returns.
  *   - Work is queued on `stream` (a cudaStream_t; NULL is the legacy default stream)
  *     and runs asynchronously; results are valid once the stream has been
  *     synchronized. Calls on the same stream run in order.
@@ -67,7 +68,8 @@ typedef enum {
     KVQ_ERR_MISALIGNED = 2,  /* a pointer below the alignment stated above */
     KVQ_ERR_UNSUPPORTED = 3, /* a size beyond what the kernels index (see each call) */
     KVQ_ERR_CAPACITY = 4,    /* a cache range past capacity_rows */
-    KVQ_ERR_CUDA = 5         /* a CUDA runtime error while queuing work */
+    KVQ_ERR_CUDA = 5,        /* a CUDA runtime error while queuing work */
+    KVQ_ERR_TIMEOUT = 6      /* a bounded wait inside a kernel gave up (kvq_device_status) */
 } kvq_status;
 
 /* Block-scale rule ("Configuration Parameters Reference": scale_rule). */
@@ -96,6 +98,14 @@ typedef enum {
  *            copy of *amax_in). At least one of amax_in / amax_out must be non-NULL.
  *   packed   device, uint8[n_elems / 2], 8-byte aligned. Written.
  *   scales   device, uint8[n_elems / 16] (e4m3 codes, one per block, same order). Written.
+ * When the amax is computed, amax pass and quantization run in one launch for tensors of
+ * up to about 2^25 blocks (larger ones take two): the tiles of the amax pass fold their
+ * maxima into *amax_out, and the quantize tiles of the same launch wait for it there, so
+ * the slot holds intermediate values until the stream reaches the end of the call. Such
+ * a wait is bounded (2 s); if it gives up, the tensor's outputs are left unwritten,
+ * *amax_out is set to NaN and kvq_device_status() reports KVQ_ERR_TIMEOUT. That only
+ * happens when the launch cannot get its CTAs onto the GPU, e.g. another stream holds
+ * every SM for longer than the bound.
  */
 kvq_status kvq_quantize(const void* x, int64_t n_elems, int32_t head_dim, kvq_scale_rule rule,
                         const float* amax_in, float* amax_out, uint8_t* packed, uint8_t* scales,
@@ -119,11 +129,24 @@ kvq_status kvq_dequantize(const uint8_t* packed, const uint8_t* scales, const fl
  *   xs, packed, scales  host arrays of n_tensors device pointers (as in kvq_quantize).
  *   amax_in   host array of n_tensors device pointers, or NULL: compute every amax.
  *   amax_out  host array of n_tensors device pointers, or NULL when amax_in is given.
+ *             When the amax is computed, every tensor needs its own slot (two tensors
+ *             sharing one return KVQ_ERR_INVALID_ARG).
  *   At most KVQ_MAX_BATCH tensors share a launch; more are split.
  */
 kvq_status kvq_quantize_batch(const void* const* xs, int32_t n_tensors, int64_t n_elems, int32_t head_dim,
                               kvq_scale_rule rule, const float* const* amax_in, float* const* amax_out,
                               uint8_t* const* packed, uint8_t* const* scales, kvq_stream_t stream);
+
+/*
+ * kvq_quantize_launches -- host only: the number of kernels kvq_quantize_batch (and
+ *   kvq_append_batch, kvq_quantize_dequantize) launches for n_tensors tensors of n_elems
+ *   elements: per group of KVQ_MAX_BATCH tensors, 1 when the amax is given (amax_given
+ *   != 0), else 2 (a slot clear and the one-launch amax + quantize) or 3 (clear, amax
+ *   pass, quantize) for tensors too large for one launch. For 16-byte-aligned packed
+ *   buffers; writes *launches (0 for empty tensors).
+ */
+kvq_status kvq_quantize_launches(int32_t n_tensors, int64_t n_elems, int32_t head_dim, int32_t amax_given,
+                                 int32_t* launches);
 
 /*
  * kvq_dequantize_batch -- n_tensors independent kvq_dequantize calls of the same size in
@@ -395,6 +418,18 @@ const char* kvq_last_error(void);
 
 /* Library version, e.g. "0.1.0". */
 const char* kvq_version(void);
+
+/*
+ * kvq_device_status -- errors that kernels of this library raised on the current device
+ *   since the last clearing call: KVQ_ERR_TIMEOUT when a bounded wait inside a kernel gave
+ *   up (see kvq_quantize), else KVQ_OK. The word is sticky and per device; clear != 0
+ *   resets it. This call copies from the device, so it waits for the device's preceding
+ *   work on the legacy default stream (and, with that stream's usual semantics, for the
+ *   work it synchronizes with); call it after synchronizing the streams of interest.
+ *   Returns KVQ_ERR_CUDA if the copy fails. kvq_attention reports its own timeouts
+ *   through its status argument instead.
+ */
+kvq_status kvq_device_status(int32_t clear);
 
 #ifdef __cplusplus
 }

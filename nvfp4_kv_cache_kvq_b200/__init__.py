@@ -19,7 +19,7 @@ from . import build as _build
 BLOCK = 16
 RULES = {"static_6": 0, "static_4": 1, "mse": 2}
 STATUS = {0: "KVQ_OK", 1: "KVQ_ERR_INVALID_ARG", 2: "KVQ_ERR_MISALIGNED", 3: "KVQ_ERR_UNSUPPORTED",
-          4: "KVQ_ERR_CAPACITY", 5: "KVQ_ERR_CUDA"}
+          4: "KVQ_ERR_CAPACITY", 5: "KVQ_ERR_CUDA", 6: "KVQ_ERR_TIMEOUT"}
 MAX_BATCH = 64
 
 _lib = None
@@ -75,6 +75,7 @@ def load() -> ctypes.CDLL:
         "kvq_attention": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, ctypes.c_uint64, P, P],
         "kvq_attention_workspace_bytes": [I32, I32, I64, U64P],
         "kvq_attention_launches": [I32, I32, I64, ctypes.POINTER(ctypes.c_int32)],
+        "kvq_quantize_launches": [I32, I64, I32, I32, ctypes.POINTER(ctypes.c_int32)],
         "kvq_attention_noalloc": [P, I32, I32, CP, CP, I64, ctypes.c_float, P, P, P],
         "kvq_recent_append_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
         "kvq_recent_read_batch": [ctypes.POINTER(_RecentCache), I32, I64, ctypes.POINTER(P), P],
@@ -89,6 +90,9 @@ def load() -> ctypes.CDLL:
     lib.kvq_status_string.argtypes, lib.kvq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
     lib.kvq_last_error.argtypes, lib.kvq_last_error.restype = [], ctypes.c_char_p
     lib.kvq_version.argtypes, lib.kvq_version.restype = [], ctypes.c_char_p
+    lib.kvq_device_status.argtypes, lib.kvq_device_status.restype = [I32], ctypes.c_int
+    lib.kvq_testing_set_fused_wait.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
+    lib.kvq_testing_set_fused_wait.restype = None
     _lib = lib
     return lib
 
@@ -122,6 +126,27 @@ def kvq_status_string(status: int) -> str:
 
 def kvq_version() -> str:
     return load().kvq_version().decode()
+
+
+def kvq_quantize_launches(n_tensors: int, n_elems: int, head_dim: int = 128, amax_given: bool = False) -> int:
+    """Kernels one quantize or append call launches (host only)."""
+    out = ctypes.c_int32()
+    _check(load().kvq_quantize_launches(int(n_tensors), int(n_elems), int(head_dim), 1 if amax_given else 0,
+                                        ctypes.byref(out)))
+    return out.value
+
+
+def kvq_device_status(clear: bool = True) -> None:
+    """Raise KvqError(KVQ_ERR_TIMEOUT) if a bounded wait inside one of the library's
+    kernels gave up on the current device since the last clearing call (the word is
+    cleared when ``clear``). Synchronize the streams of interest first."""
+    _check(load().kvq_device_status(1 if clear else 0))
+
+
+def testing_set_fused_wait(extra_a_tiles: int, wait_ns: int = 0) -> None:
+    """Test hook (kvq_testing.h): make the one-launch quantize of this thread wait for
+    amax tiles that never come, with the given bound. (0, 0) restores normal operation."""
+    load().kvq_testing_set_fused_wait(int(extra_a_tiles), int(wait_ns))
 
 
 def kvq_quantize(x: torch.Tensor, head_dim: int | None = None, rule="static_6", amax_in: torch.Tensor | None = None,
@@ -378,12 +403,15 @@ def kvq_attention_launches(n_queries: int, heads: int, n_keys: int) -> int:
 def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: int,
                   softmax_scale: float | None = None, out: torch.Tensor | None = None,
                   workspace: torch.Tensor | None = None, status: torch.Tensor | None = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, check: bool = False) -> torch.Tensor:
     """softmax(scale * Q K^T) V per head over cache tokens [0, n_keys), K and V read from
     their packed caches. q: bf16 [n_queries, heads, 128]; returns bf16 of q's shape.
     ``workspace`` (uint8, device) holds key-split partials; None allocates the size
     kvq_attention_workspace_bytes recommends, an empty tensor forbids splitting.
-    ``status`` (int32, one element, device) is set to 1 if an on-chip wait timed out."""
+    ``status`` (int32, one element, device) is set to 1 if an on-chip wait timed out; the
+    output is then invalid. The call stays asynchronous and does not read ``status``
+    unless ``check`` is set: then it synchronizes the stream and raises
+    KvqError(KVQ_ERR_TIMEOUT) when the status is nonzero."""
     if q.dim() != 3:
         raise ValueError("q must be [n_queries, heads, head_dim]")
     n_q, heads, d = q.shape
@@ -401,7 +429,19 @@ def kvq_attention(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: i
     _check(load().kvq_attention(_dev(q, "q"), n_q, heads, ctypes.byref(kc), ctypes.byref(vc), int(n_keys),
                                 float(softmax_scale), _dev(out, "out"), ws_ptr, workspace.numel(),
                                 _dev(status, "status"), _stream(stream, q.device)))
+    if check:
+        _check_status(status, stream, q.device)
     return out
+
+
+def _check_status(status: torch.Tensor, stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    if hasattr(s, "synchronize"):
+        s.synchronize()
+    else:
+        torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise KvqError(6, "an on-chip wait of the attention kernel gave up; the output is invalid")
 
 
 def kvq_attention_noalloc(q: torch.Tensor, k_cache: KVCache, v_cache: KVCache, n_keys: int,

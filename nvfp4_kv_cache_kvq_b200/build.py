@@ -9,7 +9,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SOURCES = [os.path.join(PKG, "csrc", f) for f in ("kvq.cu", "kvq_rtn.cu", "kvq_layout.cu", "kvq_attention.cu", "kvq_recent.cu")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", "kvq_device.cuh"), os.path.join(PKG, "csrc", "kvq_common.h"),
-                  os.path.join(ROOT, "include", "kvq.h")]
+                  os.path.join(ROOT, "include", "kvq.h"),
+                  os.path.join(ROOT, "include", "kvq_testing.h")]
 LIB = os.path.join(PKG, "_build", "libkvq.so")
 
 NVCC_FLAGS = [

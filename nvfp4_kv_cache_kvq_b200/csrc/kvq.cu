@@ -9,7 +9,7 @@
 //
 // Kernels (streaming passes; no tensor cores, no shared-memory staging of data: every
 // access is a fully coalesced 256-bit or narrower vector access):
-//   zero_kernel      clears the amax slots a quantize is about to reduce into.
+//   fill_kernel      sets the amax slots a quantize is about to reduce into.
 //   amax_kernel      max |x| over each tensor: 256-bit loads, a max.xorsign.abs.bf16x2
 //                    tree per block, warp redux, one atomic max per CTA.
 //   quantize_kernel  UPT units of BPT blocks per thread: one 256-bit load per block,
@@ -25,11 +25,13 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
 
 #include "kvq.h"
 #include "kvq_common.h"
 #include "kvq_device.cuh"
+#include "kvq_testing.h"
 
 namespace kvq {
 
@@ -46,6 +48,7 @@ struct AmaxBatch {
 struct ZeroBatch {
     uint32_t* out[kMaxBatch];
     int n;
+    uint32_t value;  // written to every out[i]
 };
 
 struct QuantTensor {
@@ -88,12 +91,12 @@ constexpr int kAmaxIters = 4;  // blocks per thread in amax_kernel
 
 // ---------------------------------------------------------------- kernels
 
-__global__ void __launch_bounds__(64) zero_kernel(const ZeroBatch z)
+__global__ void __launch_bounds__(64) fill_kernel(const ZeroBatch z)
 {
     pdl_begin();
     int i = threadIdx.x;
     if (i < z.n)
-        *z.out[i] = 0u;
+        *z.out[i] = z.value;
 }
 
 // grid (tiles, tensors); a tile is kThreads * kAmaxIters blocks.
@@ -155,6 +158,19 @@ __device__ __forceinline__ void build_scale_tables(ScaleTables& t, float gs)
         t.inv[c] = safe_rcp(S);
     }
     __syncthreads();
+}
+
+// The same tables built by one warp for its own use (no CTA barrier).
+__device__ __forceinline__ void build_scale_tables_warp(ScaleTables& t, float gs)
+{
+    for (int c = threadIdx.x & 31; c < 128; c += 32) {
+        float v, unused;
+        e4m3x2_to_f32(static_cast<uint32_t>(c), v, unused);
+        const float S = c == 127 ? 0.0f : __fmul_rn(v, gs);
+        t.S[c] = S;
+        t.inv[c] = safe_rcp(S);
+    }
+    __syncwarp();
 }
 
 // The block's 16 bf16 values as eight fp32 pairs (element 2j low, 2j + 1 high).
@@ -302,21 +318,29 @@ __device__ __forceinline__ void bf16_from_codes(uint32_t q0, uint32_t q1, float 
     }
 }
 
-// Unit u of a tensor: blocks [u*BPT, u*BPT + BPT) clipped to n_blocks.
-template <int RULE, int BPT, bool MARK, int MODE>
-__device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, uint64_t n_blocks,
-                                              const Quotients& qt, const ScaleTables& tab)
+// The input of unit u of a tensor: blocks [u*BPT, u*BPT + BPT) clipped to n_blocks (a
+// pair unit whose second block is past the end loads one).
+template <int BPT>
+__device__ __forceinline__ void load_unit(const QuantTensor& T, uint64_t u, uint64_t n_blocks, uint32_t (&w)[2][8])
 {
     const char* x = static_cast<const char*>(T.x);
+    const uint64_t b0 = u * BPT;
+    ld_nc_v8(x + b0 * 32, w[0]);
+    if (BPT == 2 && b0 + 1 < n_blocks)
+        ld_nc_v8(x + b0 * 32 + 32, w[1]);
+}
+
+// Quantize unit u from its loaded input w: codes, scales and (MODE) the bf16 round trip.
+template <int RULE, int BPT, bool MARK, int MODE>
+__device__ __forceinline__ void quantize_loaded(const QuantTensor& T, uint64_t u, uint64_t n_blocks,
+                                                const Quotients& qt, const ScaleTables& tab, const uint32_t (&w)[2][8])
+{
     char* y = static_cast<char*>(T.y);
     const uint64_t b0 = u * BPT;
     if (BPT == 2 && b0 + 1 < n_blocks) {
-        uint32_t w0[8], w1[8];
-        ld_nc_v8(x + b0 * 32, w0);
-        ld_nc_v8(x + b0 * 32 + 32, w1);
         uint32_t q0, q1, q2, q3;
-        const uint32_t c0 = quantize_block<RULE, MARK>(w0, qt, tab, q0, q1);
-        const uint32_t c1 = quantize_block<RULE, MARK>(w1, qt, tab, q2, q3);
+        const uint32_t c0 = quantize_block<RULE, MARK>(w[0], qt, tab, q0, q1);
+        const uint32_t c1 = quantize_block<RULE, MARK>(w[1], qt, tab, q2, q3);
         if (MODE != kYOnly) {
             st_v4(T.packed + b0 * 8, q0, q1, q2, q3);
             *reinterpret_cast<uint16_t*>(T.scales + b0) = static_cast<uint16_t>(c0 | (c1 << 8));
@@ -329,10 +353,8 @@ __device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, 
             st_v8(y + b0 * 32 + 32, yy);
         }
     } else {  // BPT == 1, or the odd last block of a pair unit
-        uint32_t w0[8];
-        ld_nc_v8(x + b0 * 32, w0);
         uint32_t q0, q1;
-        const uint32_t c0 = quantize_block<RULE, MARK>(w0, qt, tab, q0, q1);
+        const uint32_t c0 = quantize_block<RULE, MARK>(w[0], qt, tab, q0, q1);
         if (MODE != kYOnly) {
             st_v2(T.packed + b0 * 8, q0, q1);
             T.scales[b0] = static_cast<uint8_t>(c0);
@@ -345,12 +367,49 @@ __device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, 
     }
 }
 
-// grid (tiles, tensors), UPT units of BPT blocks per thread. The tiles and tensors are
-// walked in the reverse of amax_kernel's order, so the data amax_kernel read last (still
-// in L2) is quantized first. With BPT = 2 the packed pointer must be 16-byte and the
-// scale pointer 2-byte aligned. MODE selects the outputs (QuantMode); the round trip
-// y = bf16_rne(value * S) is the same arithmetic as dequant_kernel, so it is bit-equal
-// to quantizing and then dequantizing.
+// Unit u of a tensor, loaded and quantized.
+template <int RULE, int BPT, bool MARK, int MODE>
+__device__ __forceinline__ void quantize_unit(const QuantTensor& T, uint64_t u, uint64_t n_blocks,
+                                              const Quotients& qt, const ScaleTables& tab)
+{
+    uint32_t w[2][8];
+    load_unit<BPT>(T, u, n_blocks, w);
+    quantize_loaded<RULE, BPT, MARK, MODE>(T, u, n_blocks, qt, tab, w);
+}
+
+// The global scale of a tensor amax and how its block-scale quotients are computed.
+__device__ __forceinline__ Quotients make_quotients(float amax)
+{
+    Quotients qt;
+    qt.gs = __fdiv_rn(amax, kGlobalDen);
+    qt.markstein = qt.gs >= 0x1p-80f && qt.gs <= 0x1p125f;
+    qt.inv_gs = qt.markstein ? __frcp_rn(qt.gs) : 0.0f;
+    return qt;
+}
+
+// Units u0, u0 + kThreads, ... (n_units of them, stopping at the tensor's end) of one
+// thread, BPT blocks each. MARK is uniform per tensor, so each path holds one quotient
+// form only.
+template <int RULE, int BPT, int MODE, bool MARK>
+__device__ __forceinline__ void quantize_units(const QuantTensor& T, uint64_t u0, int n_units, uint64_t n_blocks,
+                                               const Quotients& qt, const ScaleTables& tab)
+{
+#pragma unroll 1
+    for (int i = 0; i < n_units; ++i) {
+        const uint64_t u = u0 + static_cast<uint64_t>(i) * kThreads;
+        if (u * BPT >= n_blocks)
+            return;
+        quantize_unit<RULE, BPT, MARK, MODE>(T, u, n_blocks, qt, tab);
+    }
+}
+
+// grid (tiles, tensors), UPT units of BPT blocks per thread; the amax of every tensor is
+// already known (the caller's amax_in, or a separate amax pass). The tiles and tensors
+// are walked in the reverse of amax_kernel's order, so the data amax_kernel read last
+// (still in L2) is quantized first. With BPT = 2 the packed pointer must be 16-byte and
+// the scale pointer 2-byte aligned. MODE selects the outputs (QuantMode); the round trip
+// y = bf16_rne(value * S) is the same arithmetic as dequant_kernel, so it is bit-equal to
+// quantizing and then dequantizing.
 template <int RULE, int BPT, int MODE, int UPT = 1>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
 {
@@ -358,25 +417,254 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const QuantBatch B)
     __shared__ ScaleTables tab;
     const QuantTensor& T = B.t[gridDim.y - 1 - blockIdx.y];
     const float amax = __ldg(T.amax);
-    Quotients qt;
-    qt.gs = __fdiv_rn(amax, kGlobalDen);
-    qt.markstein = qt.gs >= 0x1p-80f && qt.gs <= 0x1p125f;
-    qt.inv_gs = qt.markstein ? __frcp_rn(qt.gs) : 0.0f;
+    const Quotients qt = make_quotients(amax);
     if (T.amax_copy != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
         *T.amax_copy = amax;
     build_scale_tables(tab, qt.gs);
+    const uint64_t u0 = static_cast<uint64_t>(gridDim.x - 1 - blockIdx.x) * (kThreads * UPT) + threadIdx.x;
+    if (qt.markstein)
+        quantize_units<RULE, BPT, MODE, true>(T, u0, UPT, B.n_blocks, qt, tab);
+    else
+        quantize_units<RULE, BPT, MODE, false>(T, u0, UPT, B.n_blocks, qt, tab);
+}
 
-    // the CTA's tile: UPT rows of kThreads consecutive units
-    const uint64_t tile = static_cast<uint64_t>(gridDim.x - 1 - blockIdx.x) * (kThreads * UPT);
+// ---------------------------------------------------------------- device error word
+
+// Sticky per-device error word: a kernel whose bounded wait gave up ORs a bit into it;
+// kvq_device_status() reads and clears it. It is the only state the codec kernels keep.
+__device__ unsigned int g_device_error;
+constexpr unsigned kDeviceErrWaitTimeout = 1u;
+
+// ---------------------------------------------------------------- one-launch amax + quantize
+//
+// fused_quantize_kernel computes every tensor's amax and quantizes the tensor in the same
+// launch, so a tensor that fits in L2 is read from DRAM once: the quantize pass reads it
+// back from L2. Each tensor is cut into tiles of kTileBlocks blocks. The launch runs a
+// fixed sequence of tickets; ticket j holds
+//   an amax part: tile j of the amax order (tensor-major), if j < n * tiles, and
+//   a quantize part: tile j - D of the quantize order (same order), if that exists,
+// so a tensor's quantize tiles trail its amax tiles by D >= tiles tickets (a grid's
+// worth more when the job spans several waves: its amax is then mostly complete before
+// anyone asks for it, and the D tiles in flight stay in L2). CTA b takes tickets b, b + G, ...
+// in order (G = gridDim.x, at most the CTAs the GPU holds at once), so every ticket
+// before a waiting one belongs to a CTA that is running or done.
+//
+// Within a ticket: thread 0 waits for the quantize tensor's amax; a CTA barrier hands it
+// to every thread; thread 0 starts a TMA bulk copy of the amax tile into shared memory;
+// the CTA quantizes its quantize tile (the copy lands meanwhile); then each warp reduces
+// its share of the amax tile, and the last warp to finish (a shared-memory count) folds
+// the tile max into the tensor's slot. Amax parts never wait on other CTAs.
+//
+// The synchronisation lives in the caller's amax slot, so the launch needs no memory of
+// its own. fill_kernel sets the slot to kSlotBase before the launch; then
+//   bits 16..31  max |x| so far, as bf16 bits. Every |x| is a bf16 value, so the fp32 amax
+//                has zero low bits and the high half is all of it;
+//   bits  0..15  kSlotBase + the number of amax tiles folded in (below 0x7F7F, so read as a
+//                bf16 it is non-negative and finite, and the max below leaves it alone).
+// A tile folds its max into the high half (bf16 max; the low lane against +0) and then
+// adds 1, both read-modify-writes of the same word by one thread, so each count covers
+// its max. The tile whose add completes the count stores the plain fp32 amax (low half
+// 0). A reader waits (bounded) until the low half is 0 or above the number of tiles,
+// then takes the high half. If a wait gives up, the reader stores a NaN in the slot,
+// raises kDeviceErrWaitTimeout, and its tile writes nothing; readers skip a NaN slot.
+
+constexpr uint32_t kWarps = kThreads / 32;
+constexpr uint32_t kTileBlocks = 1024;        // blocks of every amax and quantize tile
+constexpr uint32_t kTileBytes = kTileBlocks * 32;
+constexpr uint32_t kSlotBase = 1u;
+
+struct FusedBatch {
+    QuantTensor t[kMaxBatch];  // t.amax: the slot, set to kSlotBase before the launch
+    uint64_t n_blocks;         // blocks per tensor
+    uint64_t total;            // tickets
+    uint64_t wait_ns;          // bound of every wait
+    uint32_t n_tensors;
+    uint32_t tiles;            // tiles per tensor
+    uint32_t q_units;          // units per thread of a quantize tile: kTileBlocks / (kThreads * BPT)
+    uint32_t expect_a;         // amax tiles a reader waits for (tiles)
+    uint32_t delay;            // D
+};
+
+constexpr uint32_t kNaNBits = 0x7FC00000u;
+
+// The slot word is complete: every amax tile folded in (low half above expect_a), or
+// the plain amax left by the last one (low half 0).
+__device__ __forceinline__ bool slot_complete(uint32_t v, uint32_t expect_a)
+{
+    const uint32_t c = v & 0xFFFFu;
+    return c == 0u || c > expect_a;
+}
+
+// Thread 0 of a CTA with a quantize part of tensor t: the amax bits, or kNaNBits.
+__device__ __forceinline__ uint32_t await_amax(const FusedBatch& B, uint32_t t)
+{
+    uint32_t* slot = reinterpret_cast<uint32_t*>(const_cast<float*>(B.t[t].amax));
+    uint32_t v = ld_relaxed_u32(slot);
+    if (!slot_complete(v, B.expect_a)) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!slot_complete(v = ld_relaxed_u32(slot), B.expect_a)) {
+            if (globaltimer_ns() - t0 > B.wait_ns) {
+                st_relaxed_u32(slot, kNaNBits);
+                atomicOr(&g_device_error, kDeviceErrWaitTimeout);
+                return kNaNBits;
+            }
+            __nanosleep(64);
+        }
+    }
+    return (v & 0xFFFF0000u) == kNaNBits ? kNaNBits : (v & 0xFFFF0000u);
+}
+
+// Fold one amax tile's max m (bf16 bits) into tensor t's slot.
+__device__ __forceinline__ void fold_amax(const FusedBatch& B, uint32_t t, uint32_t m)
+{
+    uint32_t* slot = reinterpret_cast<uint32_t*>(const_cast<float*>(B.t[t].amax));
+    red_max_bf16_high(slot, m);
+    const uint32_t old = atom_add_relaxed_u32(slot, 1u);
+    if ((old & 0xFFFFu) == kSlotBase + B.expect_a - 1)  // this add completed the count
+        st_relaxed_u32(slot, old & 0xFFFF0000u);
+}
+
+// The (tensor, tile) of position i of a tensor-major tile order, advanced by a fixed step
+// without dividing.
+struct TileCursor {
+    uint32_t t, tile;
+    __device__ __forceinline__ void start(uint64_t i, uint32_t tiles)
+    {
+        t = static_cast<uint32_t>(i / tiles);
+        tile = static_cast<uint32_t>(i % tiles);
+    }
+    __device__ __forceinline__ void advance(uint32_t step_div, uint32_t step_mod, uint32_t tiles)
+    {
+        t += step_div;
+        tile += step_mod;
+        if (tile >= tiles) {
+            tile -= tiles;
+            ++t;
+        }
+    }
+};
+
+template <int RULE, int BPT, int MODE>
+__global__ void __launch_bounds__(kThreads) fused_quantize_kernel(const FusedBatch B)
+{
+    __shared__ __align__(128) uint4 stage[kTileBytes / 16];
+    __shared__ ScaleTables tab;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t amax_bcast[2];
+    __shared__ uint32_t warp_max, warps_done;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        warp_max = 0;
+        warps_done = 0;
+    }
+    pdl_begin();
+    __syncthreads();
+    const uint64_t n_tiles = static_cast<uint64_t>(B.n_tensors) * B.tiles;
+    const uint32_t G = gridDim.x, step_div = G / B.tiles, step_mod = G % B.tiles;
+    TileCursor ac, qc;
+    ac.start(blockIdx.x, B.tiles);
+    bool q_started = false;
+    Quotients qt;
+    uint32_t tab_tensor = 0xFFFFFFFFu;  // tensor whose global scale the tables hold
+    uint32_t copies = 0;                // bulk copies issued (the mbarrier's phase)
+    uint32_t peek = 0;                  // thread 0: an early read of the next quantize tensor's slot
+    bool peeked = false;                // peek holds this ticket's slot
+    int par = 0;
 #pragma unroll 1
-    for (int i = 0; i < UPT; ++i) {
-        const uint64_t u = tile + static_cast<uint64_t>(i) * kThreads + threadIdx.x;
-        if (u * BPT >= B.n_blocks)
-            return;
-        if (qt.markstein)
-            quantize_unit<RULE, BPT, true, MODE>(T, u, B.n_blocks, qt, tab);
-        else
-            quantize_unit<RULE, BPT, false, MODE>(T, u, B.n_blocks, qt, tab);
+    for (uint64_t k = blockIdx.x; k < B.total; k += G, par ^= 1) {
+        const bool has_a = k < n_tiles;
+        const bool has_q = k >= B.delay && k - B.delay < n_tiles;
+        if (has_q && !q_started) {
+            qc.start(k - B.delay, B.tiles);
+            q_started = true;
+        }
+        if (has_q && threadIdx.x == 0)
+            amax_bcast[par] = peeked && slot_complete(peek, B.expect_a) && (peek & 0xFFFF0000u) != kNaNBits
+                                  ? peek & 0xFFFF0000u
+                                  : await_amax(B, qc.t);
+        __syncthreads();  // the amax is known; the stage, tables and warp_max are free
+        uint32_t a_bytes = 0;
+        if (has_a) {
+            const uint64_t b0 = static_cast<uint64_t>(ac.tile) * kTileBlocks;
+            const uint64_t nb = B.n_blocks - b0 < kTileBlocks ? B.n_blocks - b0 : kTileBlocks;
+            a_bytes = static_cast<uint32_t>(nb * 32);
+            if (threadIdx.x == 0) {
+                fence_proxy_async_smem();
+                bulk_load(stage, static_cast<const char*>(B.t[ac.t].x) + b0 * 32, a_bytes, &bar);
+            }
+        }
+        // thread 0 reads the next quantize tensor's slot now, to find it complete later
+        if (threadIdx.x == 0) {
+            const uint64_t kn = k + G;
+            peeked = kn >= B.delay && kn - B.delay < n_tiles;
+            if (peeked) {
+                TileCursor nc = qc;
+                if (q_started)
+                    nc.advance(step_div, step_mod, B.tiles);
+                else
+                    nc.start(kn - B.delay, B.tiles);
+                peek = ld_relaxed_u32(reinterpret_cast<const uint32_t*>(B.t[nc.t].amax));
+            }
+        }
+        if (has_q) {
+            const uint32_t amax_bits = amax_bcast[par];
+            if (amax_bits != kNaNBits) {
+                if (qc.t != tab_tensor) {
+                    qt = make_quotients(__uint_as_float(amax_bits));
+                    build_scale_tables(tab, qt.gs);  // holds a CTA barrier
+                    tab_tensor = qc.t;
+                }
+                const uint64_t u0 = static_cast<uint64_t>(qc.tile) * (kThreads * B.q_units) + threadIdx.x;
+                if (qt.markstein)
+                    quantize_units<RULE, BPT, MODE, true>(B.t[qc.t], u0, B.q_units, B.n_blocks, qt, tab);
+                else
+                    quantize_units<RULE, BPT, MODE, false>(B.t[qc.t], u0, B.q_units, B.n_blocks, qt, tab);
+            }
+        }
+        if (has_a) {
+            // wait for the copy (it was issued before the quantize part, so it has landed)
+            const uint32_t phase = copies & 1u;
+            ++copies;
+            bool landed = mbar_test_parity(&bar, phase);
+            if (!landed) {
+                const uint64_t t0 = globaltimer_ns();
+                while (!(landed = mbar_test_parity(&bar, phase)) && globaltimer_ns() - t0 <= B.wait_ns)
+                    __nanosleep(32);
+            }
+            if (!landed) {  // a copy that does not land in the bound: give up on this launch
+                if (threadIdx.x == 0)
+                    atomicOr(&g_device_error, kDeviceErrWaitTimeout);
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_test_parity(&bar, phase) && globaltimer_ns() - t0 <= B.wait_ns)
+                    __nanosleep(1000);
+                return;
+            }
+            uint32_t m = 0;
+            const uint32_t n16 = a_bytes / 16;
+#pragma unroll
+            for (uint32_t i = 0; i < kTileBytes / 16 / kThreads; ++i) {
+                const uint32_t idx = threadIdx.x + i * kThreads;
+                if (idx < n16) {
+                    const uint4 v = stage[idx];
+                    m = max(m, block_absmax_bits4(v));
+                }
+            }
+            m = __reduce_max_sync(0xFFFFFFFFu, m);
+            if ((threadIdx.x & 31) == 0) {
+                atomicMax(&warp_max, m);
+                __threadfence_block();
+                if (atomicAdd(&warps_done, 1u) == kWarps - 1) {  // the last warp folds the tile
+                    __threadfence_block();
+                    const uint32_t tile_max = atomicExch(&warp_max, 0u);
+                    warps_done = 0;
+                    fold_amax(B, ac.t, tile_max);
+                }
+            }
+        }
+        ac.advance(step_div, step_mod, B.tiles);
+        if (q_started)
+            qc.advance(step_div, step_mod, B.tiles);
     }
 }
 
@@ -482,36 +770,136 @@ cudaError_t launch_quantize(kvq_scale_rule rule, int bpt, int mode, uint64_t uni
     return launch_quantize_bpt<KVQ_RULE_MSE>(bpt, mode, units, n, qb, s);
 }
 
+// Test hook (kvq_testing.h): extra A arrivals a Q-ticket waits for, and its wait bound.
+thread_local uint32_t g_test_extra_a = 0;
+thread_local uint64_t g_test_wait_ns = 0;
+
+constexpr uint64_t kFusedWaitNs = 2000000000ull;  // 2 s
+constexpr uint64_t kFusedMaxBlocks = 2ull << 20;  // 64 MiB of bf16: larger tensors take two passes
+
+// CTAs of `kernel` the device holds at once (kThreads each), cached per device.
+template <typename Kernel>
+int resident_ctas(Kernel kernel)
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    if (dev < 64) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0)
+            return c;
+    }
+    int sms = 0, occ = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0) != cudaSuccess)
+        return 0;
+    const int r = (occ > 0 ? occ : 1) * (sms > 0 ? sms : 1);
+    if (dev < 64)
+        cache[dev].store(r, std::memory_order_relaxed);
+    return r;
+}
+
+template <int RULE, int BPT, int MODE>
+cudaError_t launch_fused(FusedBatch& fb, cudaStream_t s)
+{
+    auto kernel = fused_quantize_kernel<RULE, BPT, MODE>;
+    const int res = resident_ctas(kernel);
+    if (res <= 0)
+        return cudaErrorUnknown;
+    // quantize tiles trail their amax tiles by one tensor, plus one grid when the job
+    // spans more than one wave (two grids measured no faster and missed L2 more)
+    const uint64_t n_tiles = static_cast<uint64_t>(fb.n_tensors) * fb.tiles;
+    fb.delay = fb.tiles + (n_tiles > static_cast<uint64_t>(res) ? static_cast<uint32_t>(res) : 0u);
+    fb.total = n_tiles + fb.delay;
+    fb.q_units = kTileBlocks / (kThreads * BPT);
+    const uint64_t grid = fb.total < static_cast<uint64_t>(res) ? fb.total : static_cast<uint64_t>(res);
+    return launch(kernel, dim3(static_cast<unsigned>(grid)), kThreads, s, fb);
+}
+
+template <int RULE, int BPT>
+cudaError_t launch_fused_mode(int mode, FusedBatch& fb, cudaStream_t s)
+{
+    if (mode == kCodes)
+        return launch_fused<RULE, BPT, kCodes>(fb, s);
+    if (mode == kCodesAndY)
+        return launch_fused<RULE, BPT, kCodesAndY>(fb, s);
+    return launch_fused<RULE, BPT, kYOnly>(fb, s);
+}
+
+template <int RULE>
+cudaError_t launch_fused_bpt(int bpt, int mode, FusedBatch& fb, cudaStream_t s)
+{
+    return bpt == 2 ? launch_fused_mode<RULE, 2>(mode, fb, s) : launch_fused_mode<RULE, 1>(mode, fb, s);
+}
+
+// The one-launch plan for n tensors of n_blocks blocks, or false for tensors larger than
+// kFusedMaxBlocks (their second read would not come from L2 anyway).
+bool plan_fused(uint64_t n_blocks, int n, FusedBatch& fb)
+{
+    if (n_blocks == 0 || n_blocks > kFusedMaxBlocks)
+        return false;
+    fb.n_blocks = n_blocks;
+    fb.n_tensors = static_cast<uint32_t>(n);
+    fb.tiles = static_cast<uint32_t>((n_blocks + kTileBlocks - 1) / kTileBlocks);
+    fb.expect_a = fb.tiles + g_test_extra_a;
+    fb.wait_ns = g_test_wait_ns ? g_test_wait_ns : kFusedWaitNs;
+    return kSlotBase + fb.expect_a < 0x7F00u;
+}
+
 // Quantize a batch of equally sized tensors whose amax slots are given. When
-// compute_amax, the slots are cleared and reduced first.
+// compute_amax, the amax is reduced into the slots first: in the same launch
+// (fused_quantize_kernel) for tensors of up to kFusedMaxBlocks blocks, else by
+// amax_kernel before quantize_kernel.
 kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s,
                         int mode = kCodes)
 {
     if (n == 0 || qb.n_blocks == 0)
         return KVQ_OK;
-    kvq_status st;
-    if (compute_amax) {
-        ZeroBatch z{};
-        AmaxBatch ab{};
-        for (int i = 0; i < n; ++i) {
-            z.out[i] = reinterpret_cast<uint32_t*>(const_cast<float*>(qb.t[i].amax));
-            ab.x[i] = qb.t[i].x;
-            ab.out[i] = z.out[i];
-        }
-        z.n = n;
-        ab.n_blocks = qb.n_blocks;
-        if ((st = launched(launch(zero_kernel, dim3(1), 64, s, z), "zero_kernel")) != KVQ_OK)
-            return st;
-        if ((st = launched(launch(amax_kernel, dim3(tiles(qb.n_blocks, kAmaxIters), n), kThreads, s, ab),
-                           "amax_kernel")) != KVQ_OK)
-            return st;
-    }
     bool pairs = true;
     if (mode != kYOnly)
         for (int i = 0; i < n; ++i)
             pairs = pairs && aligned(qb.t[i].packed, 16) && aligned(qb.t[i].scales, 2);
+    const int bpt = pairs ? 2 : 1;
+    kvq_status st;
+    if (compute_amax) {
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < i; ++j)
+                if (qb.t[i].amax == qb.t[j].amax)
+                    return fail(KVQ_ERR_INVALID_ARG, "tensors %d and %d share one amax output", j, i);
+        FusedBatch fb;
+        const bool fused = plan_fused(qb.n_blocks, n, fb);
+        ZeroBatch z{};
+        for (int i = 0; i < n; ++i)
+            z.out[i] = reinterpret_cast<uint32_t*>(const_cast<float*>(qb.t[i].amax));
+        z.n = n;
+        z.value = fused ? kSlotBase : 0u;
+        if ((st = launched(launch(fill_kernel, dim3(1), 64, s, z), "fill_kernel")) != KVQ_OK)
+            return st;
+        if (fused) {
+            for (int i = 0; i < n; ++i)
+                fb.t[i] = qb.t[i];
+            cudaError_t e;
+            if (rule == KVQ_RULE_STATIC_6)
+                e = launch_fused_bpt<KVQ_RULE_STATIC_6>(bpt, mode, fb, s);
+            else if (rule == KVQ_RULE_STATIC_4)
+                e = launch_fused_bpt<KVQ_RULE_STATIC_4>(bpt, mode, fb, s);
+            else
+                e = launch_fused_bpt<KVQ_RULE_MSE>(bpt, mode, fb, s);
+            return launched(e, "fused_quantize_kernel");
+        }
+        AmaxBatch ab{};
+        for (int i = 0; i < n; ++i) {
+            ab.x[i] = qb.t[i].x;
+            ab.out[i] = z.out[i];
+        }
+        ab.n_blocks = qb.n_blocks;
+        if ((st = launched(launch(amax_kernel, dim3(tiles(qb.n_blocks, kAmaxIters), n), kThreads, s, ab),
+                           "amax_kernel")) != KVQ_OK)
+            return st;
+    }
     const uint64_t units = pairs ? (qb.n_blocks + 1) / 2 : qb.n_blocks;
-    return launched(launch_quantize(rule, pairs ? 2 : 1, mode, units, n, qb, s), "quantize_kernel");
+    return launched(launch_quantize(rule, bpt, mode, units, n, qb, s), "quantize_kernel");
 }
 
 // Dequantize blocks [blk_lo, blk_hi) of n equally laid-out tensors; packed/scales point at
@@ -563,12 +951,6 @@ kvq_status check_cache(const kvq_cache* c, const char* what)
 }
 
 }  // namespace kvq
-
-using namespace kvq;
-
-extern "C" {
-
-}  // extern "C"
 
 namespace kvq {
 
@@ -681,6 +1063,8 @@ kvq_status dequantize_impl(const uint8_t* const* packed, const uint8_t* const* s
 }
 
 }  // namespace kvq
+
+using namespace kvq;
 
 extern "C" {
 
@@ -890,11 +1274,52 @@ const char* kvq_status_string(kvq_status status)
     case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
     case KVQ_ERR_CAPACITY: return "KVQ_ERR_CAPACITY";
     case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+    case KVQ_ERR_TIMEOUT: return "KVQ_ERR_TIMEOUT";
     }
     return "KVQ_ERR_UNKNOWN";
 }
 
 const char* kvq_last_error(void) { return g_last_error; }
+
+kvq_status kvq_quantize_launches(int32_t n_tensors, int64_t n_elems, int32_t head_dim, int32_t amax_given,
+                                 int32_t* launches)
+{
+    kvq_status st;
+    if ((st = check_shape(n_elems, head_dim)) != KVQ_OK)
+        return st;
+    if (n_tensors < 0 || launches == nullptr)
+        return fail(KVQ_ERR_INVALID_ARG, "kvq_quantize_launches: negative tensor count or null output");
+    const uint64_t n_blocks = static_cast<uint64_t>(n_elems) / kBlock;
+    const int32_t groups = (n_tensors + kMaxBatch - 1) / kMaxBatch;
+    FusedBatch fb;
+    const int32_t per = n_blocks == 0 ? 0 : amax_given ? 1 : plan_fused(n_blocks, 1, fb) ? 2 : 3;
+    *launches = groups * per;
+    return ok();
+}
+
+kvq_status kvq_device_status(int32_t clear)
+{
+    NvtxRange nvtx_range("kvq_device_status");
+    unsigned int word = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word));
+    if (e == cudaSuccess && clear && word != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(KVQ_ERR_CUDA, "kvq_device_status: %s", cudaGetErrorString(e));
+    }
+    if (word & kDeviceErrWaitTimeout)
+        return fail(KVQ_ERR_TIMEOUT, "a kernel's bounded wait for the amax of its tensor gave up");
+    return ok();
+}
+
+void kvq_testing_set_fused_wait(uint32_t extra_a_tiles, uint64_t wait_ns)
+{
+    g_test_extra_a = extra_a_tiles;
+    g_test_wait_ns = wait_ns;
+}
 
 const char* kvq_version(void) { return "0.1.0"; }
 

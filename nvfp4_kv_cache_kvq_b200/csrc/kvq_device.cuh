@@ -81,6 +81,13 @@ __device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&w)[8])
     return max(m & 0xFFFFu, m >> 16);
 }
 
+// |x| max of eight bf16 values (a 16-byte vector), as the bf16 bit pattern (sign cleared).
+__device__ __forceinline__ uint32_t block_absmax_bits4(const uint4& v)
+{
+    const uint32_t m = absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w)) & 0x7FFF7FFFu;
+    return max(m & 0xFFFFu, m >> 16);
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic): the low 32 bits hold the first value.
 __device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi)
 {
@@ -228,6 +235,104 @@ __device__ __forceinline__ uint32_t bf16x2_from_f32(float hi, float lo)
     uint32_t d;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
     return d;
+}
+
+}  // namespace kvq
+
+namespace kvq {
+
+// ---- device-scope atomics and waits on one 32-bit word (relaxed: the word itself
+// carries every value another CTA needs, so no other memory is ordered by them)
+
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u32(uint32_t* p, uint32_t v)
+{
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t atom_add_relaxed_u32(uint32_t* p, uint32_t v)
+{
+    uint32_t old;
+    asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void red_add_relaxed_u32(uint32_t* p, uint32_t v)
+{
+    asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Lane-wise bf16 max on the two 16-bit halves of *p: the low half with +0, the high half
+// with m (bf16 bits). No flush to zero, so a non-negative low half (any value up to
+// 0x7F7F read as bf16) is left exactly as it was.
+__device__ __forceinline__ void red_max_bf16_high(uint32_t* p, uint32_t m)
+{
+    const uint16_t lo = 0, hi = static_cast<uint16_t>(m);
+    asm volatile("red.relaxed.gpu.global.v2.bf16.max.noftz [%0], {%1, %2};" ::"l"(p), "h"(lo), "h"(hi) : "memory");
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+}  // namespace kvq
+
+namespace kvq {
+
+// ---- one-dimensional TMA bulk copy into this CTA's shared memory, completed on an mbarrier
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Order this thread's earlier generic-proxy accesses of shared memory before later
+// async-proxy (TMA) accesses, and make an mbarrier init visible to the async proxy.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// bytes (a multiple of 16, both addresses 16-byte aligned) from global src to shared dst;
+// the mbarrier's current phase completes when they have landed.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test_parity(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done)
+                 : "r"(smem_addr(bar)), "r"(parity)
+                 : "memory");
+    return done != 0;
 }
 
 }  // namespace kvq

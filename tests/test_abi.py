@@ -11,20 +11,24 @@ import pytest
 import nvfp4_kv_cache_kvq_b200 as kvq
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "kvq.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(kvq_\w+)\s*\(", src, flags=re.M)))
+    names = set()
+    for h in HEADERS:
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(kvq_\w+)\s*\(", src, flags=re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
     names = declared_functions()
     for must in ("kvq_quantize", "kvq_dequantize", "kvq_quantize_batch", "kvq_dequantize_batch",
                  "kvq_quantize_dequantize", "kvq_append", "kvq_append_batch", "kvq_dequantize_cache",
-                 "kvq_dequantize_cache_batch", "kvq_cache_bytes", "kvq_status_string", "kvq_last_error"):
+                 "kvq_dequantize_cache_batch", "kvq_cache_bytes", "kvq_status_string", "kvq_last_error",
+                 "kvq_device_status", "kvq_testing_set_fused_wait"):
         assert must in names
 
 
@@ -48,6 +52,7 @@ def test_library_is_built_for_sm100a_only():
 def test_host_only_calls():
     assert kvq.kvq_status_string(0) == "KVQ_OK"
     assert kvq.kvq_status_string(4) == "KVQ_ERR_CAPACITY"
+    assert kvq.kvq_status_string(6) == "KVQ_ERR_TIMEOUT"
     assert kvq.kvq_version().count(".") == 2
     p, s, a = kvq.kvq_cache_bytes(30, 12, 93600, 128, 1560)
     elems = 60 * 93600 * 12 * 128
@@ -88,6 +93,10 @@ def test_invalid_arguments_rejected_before_any_launch():
     outs = (ctypes.c_void_p * 2)(A, A)
     assert lib.kvq_quantize_batch(xs, 2, 128, 128, 0, ain, None, outs, outs, None) == 1
     assert lib.kvq_quantize_batch(xs, -1, 128, 128, 0, None, outs, outs, outs, None) == 1
+    # computed amax: two tensors may not share one amax output (the slot is the launch's
+    # synchronisation word)
+    assert lib.kvq_quantize_batch(xs, 2, 128, 128, 2, None, outs, outs, outs, None) == 1
+    assert b"share one amax output" in lib.kvq_last_error()
 
 
 def _cache(capacity_rows=64, rows_per_chunk=16, head_dim=128, base=1 << 40):
@@ -108,6 +117,15 @@ def test_append_capacity_and_alignment_checked_on_host():
     y = _fake(1 << 42)
     assert lib.kvq_dequantize_cache(ctypes.byref(c), 0, 65, y, None) == 4
     assert lib.kvq_dequantize_cache(ctypes.byref(c), 10, 5, y, None) == 1
+
+
+def test_append_batch_rejects_a_shared_chunk_amax():
+    lib = kvq.load()
+    arr = (kvq._Cache * 2)(_cache(), _cache())
+    offs = (ctypes.c_int64 * 2)(16, 16)  # same caches' buffers, same chunk: one amax slot
+    ptrs = (ctypes.c_void_p * 2)(1 << 41, 1 << 42)
+    assert lib.kvq_append_batch(arr, offs, ptrs, 2, 16, 2, None) == 1
+    assert b"share one amax output" in lib.kvq_last_error()
 
 
 def test_batch_rejects_mixed_head_dims():

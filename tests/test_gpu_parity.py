@@ -40,6 +40,27 @@ def test_worked_example_on_gpu(rule):
     assert_same(y, floats_to_bf16_bits(g[f"{rule}.dequant"]), "dequant")
 
 
+def test_mse_near_tie_blocks_on_gpu(orc):
+    """The hand-worked near-tie blocks, whose choice depends on the order of the error
+    sum: as given, then tiled over many CTAs, through quantize and through append."""
+    g = read_sections("mse_near_ties.txt")
+    x = floats_to_bf16_bits(g["input"])
+    p, s, a, y = gpu_round_trip(_bf16(x), "mse", 16)
+    assert a == float(g["amax"][0])
+    assert_same(s, hex_bytes(g["fma_even_odd.scales"]), "scales")
+    assert_same(p, hex_bytes(g["fma_even_odd.packed"]), "packed")
+    big = np.tile(x, 4096)  # 1536 rows of 128
+    check_full(orc, _bf16(big), "mse", 128)
+    rows = big.size // 128
+    cache = kvq.allocate_caches(1, 1, rows, 128, rows, "cuda")[0]
+    kvq.kvq_append(cache, 0, _bf16(big).view(rows, 128), "mse")
+    torch.cuda.synchronize()
+    pe, se, ae = orc.quantize(big, 128, "mse")
+    assert float(cache.amax.cpu()[0]) == ae
+    assert_same(cache.scales.cpu().numpy(), se, "append scales")
+    assert_same(cache.packed.cpu().numpy(), pe, "append packed")
+
+
 @pytest.mark.parametrize("rule", RULES)
 def test_single_k(orc, rule):
     """[4096, 128] N(0,1), seed 0."""

@@ -88,6 +88,8 @@ struct DequantBatch {
 // window of memory. On B200 this measured 10-15% more DRAM throughput than a
 // persistent grid-stride loop over the same bytes.
 constexpr int kAmaxIters = 4;  // blocks per thread in amax_kernel
+constexpr int kQWarps = kThreads / 32 - 1;  // quantize warps of fused_quantize_kernel (one warp reduces amax)
+constexpr int kQThreads = kQWarps * 32;
 
 // ---------------------------------------------------------------- kernels
 
@@ -387,16 +389,16 @@ __device__ __forceinline__ Quotients make_quotients(float amax)
     return qt;
 }
 
-// Units u0, u0 + kThreads, ... (n_units of them, stopping at the tensor's end) of one
+// Units u0, u0 + STRIDE, ... (n_units of them, stopping at the tensor's end) of one
 // thread, BPT blocks each. MARK is uniform per tensor, so each path holds one quotient
 // form only.
-template <int RULE, int BPT, int MODE, bool MARK>
+template <int RULE, int BPT, int MODE, bool MARK, int STRIDE = kThreads>
 __device__ __forceinline__ void quantize_units(const QuantTensor& T, uint64_t u0, int n_units, uint64_t n_blocks,
                                                const Quotients& qt, const ScaleTables& tab)
 {
 #pragma unroll 1
     for (int i = 0; i < n_units; ++i) {
-        const uint64_t u = u0 + static_cast<uint64_t>(i) * kThreads;
+        const uint64_t u = u0 + static_cast<uint64_t>(i) * STRIDE;
         if (u * BPT >= n_blocks)
             return;
         quantize_unit<RULE, BPT, MARK, MODE>(T, u, n_blocks, qt, tab);
@@ -439,21 +441,23 @@ constexpr unsigned kDeviceErrWaitTimeout = 1u;
 //
 // fused_quantize_kernel computes every tensor's amax and quantizes the tensor in the same
 // launch, so a tensor that fits in L2 is read from DRAM once: the quantize pass reads it
-// back from L2. Each tensor is cut into tiles of kTileBlocks blocks. The launch runs a
-// fixed sequence of tickets; ticket j holds
-//   an amax part: tile j of the amax order (tensor-major), if j < n * tiles, and
-//   a quantize part: tile j - D of the quantize order (same order), if that exists,
-// so a tensor's quantize tiles trail its amax tiles by D >= tiles tickets (a grid's
-// worth more when the job spans several waves: its amax is then mostly complete before
-// anyone asks for it, and the D tiles in flight stay in L2). CTA b takes tickets b, b + G, ...
-// in order (G = gridDim.x, at most the CTAs the GPU holds at once), so every ticket
-// before a waiting one belongs to a CTA that is running or done.
-//
-// Within a ticket: thread 0 waits for the quantize tensor's amax; a CTA barrier hands it
-// to every thread; thread 0 starts a TMA bulk copy of the amax tile into shared memory;
-// the CTA quantizes its quantize tile (the copy lands meanwhile); then each warp reduces
-// its share of the amax tile, and the last warp to finish (a shared-memory count) folds
-// the tile max into the tensor's slot. Amax parts never wait on other CTAs.
+// back from L2. Each tensor is cut into tiles of kTileBlocks blocks, and the tiles are
+// dealt to the CTAs round-robin in tensor-major order (CTA b takes tiles b, b + G, ...;
+// G = gridDim.x, at most the CTAs the GPU holds at once). In every CTA
+//   one warp (the amax warp) takes its tiles' amax parts: a TMA bulk copy into shared
+//   memory, a max over it, folded into the tensor's amax slot;
+//   the other kQWarps warps take the same tiles' quantize parts, each once its tensor's
+//   amax is complete, meeting among themselves at a named barrier per tile (amax
+//   broadcast, scale tables).
+// The amax warp runs ahead of its own CTA's quantize warps by at most `window` tiles (one
+// tensor and one and a half grids): far enough that a tensor's amax is mostly complete
+// before its quantize tiles ask for it, close enough that the tiles in between are still
+// in L2 when they are quantized (a global throttle, an amax warp waiting for tensor t - L
+// to be quantized everywhere, measured slower and missed L2 on most re-reads). A tensor
+// the quantize warps wait for has all its amax tiles within the reach of the CTAs that
+// own them: each of those CTAs' quantize warps is at or past that tensor, and the window
+// covers a whole tensor beyond it. So no wait depends on itself. The quantize warps share
+// nothing with the amax warp but the position they publish.
 //
 // The synchronisation lives in the caller's amax slot, so the launch needs no memory of
 // its own. fill_kernel sets the slot to kSlotBase before the launch; then
@@ -463,42 +467,50 @@ constexpr unsigned kDeviceErrWaitTimeout = 1u;
 //                bf16 it is non-negative and finite, and the max below leaves it alone).
 // A tile folds its max into the high half (bf16 max; the low lane against +0) and then
 // adds 1, both read-modify-writes of the same word by one thread, so each count covers
-// its max. The tile whose add completes the count stores the plain fp32 amax (low half
-// 0). A reader waits (bounded) until the low half is 0 or above the number of tiles,
-// then takes the high half. If a wait gives up, the reader stores a NaN in the slot,
-// raises kDeviceErrWaitTimeout, and its tile writes nothing; readers skip a NaN slot.
+// its max; neither waits for a reply. A reader waits (bounded) until the low half is 0
+// or above the number of tiles, takes the high half, and, if the low half was not 0,
+// stores the plain fp32 amax (low half 0): once every tile is in nothing else writes the
+// slot, so all readers store the same word, and every tensor has a reader. If a wait
+// gives up, the reader stores a NaN in the slot, raises kDeviceErrWaitTimeout, and its
+// tile writes nothing; readers skip a NaN slot.
 
-constexpr uint32_t kWarps = kThreads / 32;
-constexpr uint32_t kTileBlocks = 1024;        // blocks of every amax and quantize tile
+constexpr uint32_t kTileBlocks = 896;             // blocks of a tile (kQThreads x 2 units x 2 blocks)
 constexpr uint32_t kTileBytes = kTileBlocks * 32;
 constexpr uint32_t kSlotBase = 1u;
+constexpr uint32_t kQBarrier = 1;                 // named barrier of the quantize warps
 
 struct FusedBatch {
     QuantTensor t[kMaxBatch];  // t.amax: the slot, set to kSlotBase before the launch
     uint64_t n_blocks;         // blocks per tensor
-    uint64_t total;            // tickets
     uint64_t wait_ns;          // bound of every wait
     uint32_t n_tensors;
     uint32_t tiles;            // tiles per tensor
-    uint32_t q_units;          // units per thread of a quantize tile: kTileBlocks / (kThreads * BPT)
-    uint32_t expect_a;         // amax tiles a reader waits for (tiles)
-    uint32_t delay;            // D
+    uint32_t q_units;          // units per quantize thread of a tile: kTileBlocks / (kQThreads * BPT)
+    uint32_t expect_a;         // amax tiles a quantize tile waits for (tiles)
+    uint32_t window;           // tiles the amax warp may run ahead of its CTA's quantize position
+    uint32_t n_sm;             // multiprocessors of the device
 };
 
 constexpr uint32_t kNaNBits = 0x7FC00000u;
+constexpr uint32_t kQDone = 0xFFFFFFFFu;  // published quantize position: no more tiles
+
+__device__ __forceinline__ uint32_t* slot_of(const FusedBatch& B, uint32_t t)
+{
+    return reinterpret_cast<uint32_t*>(const_cast<float*>(B.t[t].amax));
+}
 
 // The slot word is complete: every amax tile folded in (low half above expect_a), or
-// the plain amax left by the last one (low half 0).
+// the plain amax left by a reader (low half 0).
 __device__ __forceinline__ bool slot_complete(uint32_t v, uint32_t expect_a)
 {
     const uint32_t c = v & 0xFFFFu;
     return c == 0u || c > expect_a;
 }
 
-// Thread 0 of a CTA with a quantize part of tensor t: the amax bits, or kNaNBits.
+// The amax bits of tensor t, or kNaNBits if the wait gave up (or an earlier one did).
 __device__ __forceinline__ uint32_t await_amax(const FusedBatch& B, uint32_t t)
 {
-    uint32_t* slot = reinterpret_cast<uint32_t*>(const_cast<float*>(B.t[t].amax));
+    uint32_t* slot = slot_of(B, t);
     uint32_t v = ld_relaxed_u32(slot);
     if (!slot_complete(v, B.expect_a)) {
         const uint64_t t0 = globaltimer_ns();
@@ -511,38 +523,76 @@ __device__ __forceinline__ uint32_t await_amax(const FusedBatch& B, uint32_t t)
             __nanosleep(64);
         }
     }
-    return (v & 0xFFFF0000u) == kNaNBits ? kNaNBits : (v & 0xFFFF0000u);
+    if ((v & 0xFFFF0000u) == kNaNBits)
+        return kNaNBits;
+    if ((v & 0xFFFFu) != 0)  // complete but not yet plain: every reader may store the same amax
+        st_relaxed_u32(slot, v & 0xFFFF0000u);
+    return v & 0xFFFF0000u;
 }
 
-// Fold one amax tile's max m (bf16 bits) into tensor t's slot.
-__device__ __forceinline__ void fold_amax(const FusedBatch& B, uint32_t t, uint32_t m)
+// The amax warp: the amax parts of tiles blockIdx.x, blockIdx.x + G, ... Each waits until
+// the CTA's quantize warps have reached within `window` of it.
+__device__ __forceinline__ void amax_warp(const FusedBatch& B, uint4* stage, uint64_t* bar, const uint32_t* q_pos)
 {
-    uint32_t* slot = reinterpret_cast<uint32_t*>(const_cast<float*>(B.t[t].amax));
-    red_max_bf16_high(slot, m);
-    const uint32_t old = atom_add_relaxed_u32(slot, 1u);
-    if ((old & 0xFFFFu) == kSlotBase + B.expect_a - 1)  // this add completed the count
-        st_relaxed_u32(slot, old & 0xFFFF0000u);
-}
-
-// The (tensor, tile) of position i of a tensor-major tile order, advanced by a fixed step
-// without dividing.
-struct TileCursor {
-    uint32_t t, tile;
-    __device__ __forceinline__ void start(uint64_t i, uint32_t tiles)
-    {
-        t = static_cast<uint32_t>(i / tiles);
-        tile = static_cast<uint32_t>(i % tiles);
-    }
-    __device__ __forceinline__ void advance(uint32_t step_div, uint32_t step_mod, uint32_t tiles)
-    {
-        t += step_div;
-        tile += step_mod;
-        if (tile >= tiles) {
-            tile -= tiles;
-            ++t;
+    const uint32_t lane = threadIdx.x & 31;
+    const uint64_t n_tiles = static_cast<uint64_t>(B.n_tensors) * B.tiles;
+    uint32_t phase = 0;
+#pragma unroll 1
+    for (uint64_t a = blockIdx.x; a < n_tiles; a += gridDim.x, phase ^= 1) {
+        uint32_t qp = ld_volatile_smem(q_pos);
+        if (qp != kQDone && a > static_cast<uint64_t>(qp) + B.window) {
+            const uint64_t t0 = globaltimer_ns();
+            while ((qp = ld_volatile_smem(q_pos)) != kQDone && a > static_cast<uint64_t>(qp) + B.window) {
+                if (globaltimer_ns() - t0 > B.wait_ns) {
+                    if (lane == 0)
+                        atomicOr(&g_device_error, kDeviceErrWaitTimeout);
+                    return;  // no copy in flight
+                }
+                __nanosleep(256);
+            }
+        }
+        const uint32_t t = static_cast<uint32_t>(a / B.tiles);
+        const uint64_t b0 = (a % B.tiles) * kTileBlocks;
+        const uint32_t nb = static_cast<uint32_t>(B.n_blocks - b0 < kTileBlocks ? B.n_blocks - b0 : kTileBlocks);
+        __syncwarp();  // every lane has read the stage of the previous tile
+        if (lane == 0) {
+            fence_proxy_async_smem();
+            bulk_load(stage, static_cast<const char*>(B.t[t].x) + b0 * 32, nb * 32, bar);
+        }
+        bool landed = mbar_test_parity(bar, phase);
+        if (!landed) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!(landed = mbar_test_parity(bar, phase)) && globaltimer_ns() - t0 <= B.wait_ns)
+                __nanosleep(32);
+        }
+        if (!landed) {  // a copy that does not land in the bound: wait once more, then leave
+            if (lane == 0)
+                atomicOr(&g_device_error, kDeviceErrWaitTimeout);
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_test_parity(bar, phase) && globaltimer_ns() - t0 <= B.wait_ns)
+                __nanosleep(1000);
+            return;
+        }
+        // lane-wise |x| maxima over the tile's 16-byte vectors, then across lanes
+        const uint32_t n16 = nb * 2;
+        uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 4
+        for (uint32_t i = lane; i < n16; i += 32) {
+            const uint4 w = stage[i];
+            m0 = absmax_bf16x2(m0, w.x);
+            m1 = absmax_bf16x2(m1, w.y);
+            m2 = absmax_bf16x2(m2, w.z);
+            m3 = absmax_bf16x2(m3, w.w);
+        }
+        uint32_t m = absmax_bf16x2(absmax_bf16x2(m0, m1), absmax_bf16x2(m2, m3)) & 0x7FFF7FFFu;
+        m = __reduce_max_sync(0xFFFFFFFFu, max(m & 0xFFFFu, m >> 16));
+        if (lane == 0) {  // fold: max into the high half, then count; no reply awaited
+            uint32_t* slot = slot_of(B, t);
+            red_max_bf16_high(slot, m);
+            red_add_relaxed_u32(slot, 1u);
         }
     }
-};
+}
 
 template <int RULE, int BPT, int MODE>
 __global__ void __launch_bounds__(kThreads) fused_quantize_kernel(const FusedBatch B)
@@ -550,122 +600,59 @@ __global__ void __launch_bounds__(kThreads) fused_quantize_kernel(const FusedBat
     __shared__ __align__(128) uint4 stage[kTileBytes / 16];
     __shared__ ScaleTables tab;
     __shared__ uint64_t bar;
-    __shared__ uint32_t amax_bcast[2];
-    __shared__ uint32_t warp_max, warps_done;
+    __shared__ uint32_t q_pos;  // the quantize warps' current tile
+    __shared__ uint32_t amax_bcast;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1);
         fence_mbar_init();
-        warp_max = 0;
-        warps_done = 0;
+        q_pos = 0;
     }
     pdl_begin();
-    __syncthreads();
-    const uint64_t n_tiles = static_cast<uint64_t>(B.n_tensors) * B.tiles;
-    const uint32_t G = gridDim.x, step_div = G / B.tiles, step_mod = G % B.tiles;
-    TileCursor ac, qc;
-    ac.start(blockIdx.x, B.tiles);
-    bool q_started = false;
-    Quotients qt;
-    uint32_t tab_tensor = 0xFFFFFFFFu;  // tensor whose global scale the tables hold
-    uint32_t copies = 0;                // bulk copies issued (the mbarrier's phase)
-    uint32_t peek = 0;                  // thread 0: an early read of the next quantize tensor's slot
-    bool peeked = false;                // peek holds this ticket's slot
-    int par = 0;
-#pragma unroll 1
-    for (uint64_t k = blockIdx.x; k < B.total; k += G, par ^= 1) {
-        const bool has_a = k < n_tiles;
-        const bool has_q = k >= B.delay && k - B.delay < n_tiles;
-        if (has_q && !q_started) {
-            qc.start(k - B.delay, B.tiles);
-            q_started = true;
-        }
-        if (has_q && threadIdx.x == 0)
-            amax_bcast[par] = peeked && slot_complete(peek, B.expect_a) && (peek & 0xFFFF0000u) != kNaNBits
-                                  ? peek & 0xFFFF0000u
-                                  : await_amax(B, qc.t);
-        __syncthreads();  // the amax is known; the stage, tables and warp_max are free
-        uint32_t a_bytes = 0;
-        if (has_a) {
-            const uint64_t b0 = static_cast<uint64_t>(ac.tile) * kTileBlocks;
-            const uint64_t nb = B.n_blocks - b0 < kTileBlocks ? B.n_blocks - b0 : kTileBlocks;
-            a_bytes = static_cast<uint32_t>(nb * 32);
-            if (threadIdx.x == 0) {
-                fence_proxy_async_smem();
-                bulk_load(stage, static_cast<const char*>(B.t[ac.t].x) + b0 * 32, a_bytes, &bar);
-            }
-        }
-        // thread 0 reads the next quantize tensor's slot now, to find it complete later
-        if (threadIdx.x == 0) {
-            const uint64_t kn = k + G;
-            peeked = kn >= B.delay && kn - B.delay < n_tiles;
-            if (peeked) {
-                TileCursor nc = qc;
-                if (q_started)
-                    nc.advance(step_div, step_mod, B.tiles);
-                else
-                    nc.start(kn - B.delay, B.tiles);
-                peek = ld_relaxed_u32(reinterpret_cast<const uint32_t*>(B.t[nc.t].amax));
-            }
-        }
-        if (has_q) {
-            const uint32_t amax_bits = amax_bcast[par];
-            if (amax_bits != kNaNBits) {
-                if (qc.t != tab_tensor) {
-                    qt = make_quotients(__uint_as_float(amax_bits));
-                    build_scale_tables(tab, qt.gs);  // holds a CTA barrier
-                    tab_tensor = qc.t;
-                }
-                const uint64_t u0 = static_cast<uint64_t>(qc.tile) * (kThreads * B.q_units) + threadIdx.x;
-                if (qt.markstein)
-                    quantize_units<RULE, BPT, MODE, true>(B.t[qc.t], u0, B.q_units, B.n_blocks, qt, tab);
-                else
-                    quantize_units<RULE, BPT, MODE, false>(B.t[qc.t], u0, B.q_units, B.n_blocks, qt, tab);
-            }
-        }
-        if (has_a) {
-            // wait for the copy (it was issued before the quantize part, so it has landed)
-            const uint32_t phase = copies & 1u;
-            ++copies;
-            bool landed = mbar_test_parity(&bar, phase);
-            if (!landed) {
-                const uint64_t t0 = globaltimer_ns();
-                while (!(landed = mbar_test_parity(&bar, phase)) && globaltimer_ns() - t0 <= B.wait_ns)
-                    __nanosleep(32);
-            }
-            if (!landed) {  // a copy that does not land in the bound: give up on this launch
-                if (threadIdx.x == 0)
-                    atomicOr(&g_device_error, kDeviceErrWaitTimeout);
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_test_parity(&bar, phase) && globaltimer_ns() - t0 <= B.wait_ns)
-                    __nanosleep(1000);
-                return;
-            }
-            uint32_t m = 0;
-            const uint32_t n16 = a_bytes / 16;
-#pragma unroll
-            for (uint32_t i = 0; i < kTileBytes / 16 / kThreads; ++i) {
-                const uint32_t idx = threadIdx.x + i * kThreads;
-                if (idx < n16) {
-                    const uint4 v = stage[idx];
-                    m = max(m, block_absmax_bits4(v));
-                }
-            }
-            m = __reduce_max_sync(0xFFFFFFFFu, m);
-            if ((threadIdx.x & 31) == 0) {
-                atomicMax(&warp_max, m);
-                __threadfence_block();
-                if (atomicAdd(&warps_done, 1u) == kWarps - 1) {  // the last warp folds the tile
-                    __threadfence_block();
-                    const uint32_t tile_max = atomicExch(&warp_max, 0u);
-                    warps_done = 0;
-                    fold_amax(B, ac.t, tile_max);
-                }
-            }
-        }
-        ac.advance(step_div, step_mod, B.tiles);
-        if (q_started)
-            qc.advance(step_div, step_mod, B.tiles);
+    __syncthreads();  // the last CTA-wide barrier: from here the amax warp and the rest run apart
+    // The amax warp's index rotates with the wave of CTAs (CTAs b and b + n_sm usually share
+    // an SM), so the amax warps of an SM sit on different sub-partitions.
+    const uint32_t warp = threadIdx.x >> 5, a_warp = (blockIdx.x / B.n_sm) & 3u;
+    if (warp == a_warp) {
+        amax_warp(B, stage, &bar, &q_pos);
+        return;
     }
+    const uint32_t qt_idx = (warp < a_warp ? warp : warp - 1) * 32 + (threadIdx.x & 31);  // 0 .. kQThreads-1
+    const uint64_t n_tiles = static_cast<uint64_t>(B.n_tensors) * B.tiles;
+    Quotients qt;
+    uint32_t tab_tensor = 0xFFFFFFFFu;
+#pragma unroll 1
+    for (uint64_t q = blockIdx.x; q < n_tiles; q += gridDim.x) {
+        const uint32_t t = static_cast<uint32_t>(q / B.tiles), tile = static_cast<uint32_t>(q % B.tiles);
+        if (qt_idx == 0) {
+            st_volatile_smem(&q_pos, static_cast<uint32_t>(q));  // publish the position, then wait
+            amax_bcast = await_amax(B, t);
+        }
+        named_barrier(kQBarrier, kQThreads);  // the amax is known; the tables are free
+        const uint32_t amax_bits = amax_bcast;
+        if (amax_bits == kNaNBits) {
+            named_barrier(kQBarrier, kQThreads);  // everyone has read amax_bcast
+            continue;
+        }
+        if (t != tab_tensor) {
+            qt = make_quotients(__uint_as_float(amax_bits));
+            for (uint32_t c = qt_idx; c < 128; c += kQThreads) {
+                float v, unused;
+                e4m3x2_to_f32(c, v, unused);
+                const float S = c == 127 ? 0.0f : __fmul_rn(v, qt.gs);
+                tab.S[c] = S;
+                tab.inv[c] = safe_rcp(S);
+            }
+            tab_tensor = t;
+        }
+        named_barrier(kQBarrier, kQThreads);  // tables ready; amax_bcast read by everyone
+        const uint64_t u0 = static_cast<uint64_t>(tile) * (kQThreads * B.q_units) + qt_idx;
+        if (qt.markstein)
+            quantize_units<RULE, BPT, MODE, true, kQThreads>(B.t[t], u0, B.q_units, B.n_blocks, qt, tab);
+        else
+            quantize_units<RULE, BPT, MODE, false, kQThreads>(B.t[t], u0, B.q_units, B.n_blocks, qt, tab);
+    }
+    if (qt_idx == 0)
+        st_volatile_smem(&q_pos, kQDone);
 }
 
 // One block: 8 code bytes and its scale code under global scale gs -> 16 bf16.
@@ -800,6 +787,15 @@ int resident_ctas(Kernel kernel)
     return r;
 }
 
+int sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+        return 1;
+    return sms > 0 ? sms : 1;
+}
+
 template <int RULE, int BPT, int MODE>
 cudaError_t launch_fused(FusedBatch& fb, cudaStream_t s)
 {
@@ -807,13 +803,14 @@ cudaError_t launch_fused(FusedBatch& fb, cudaStream_t s)
     const int res = resident_ctas(kernel);
     if (res <= 0)
         return cudaErrorUnknown;
-    // quantize tiles trail their amax tiles by one tensor, plus one grid when the job
-    // spans more than one wave (two grids measured no faster and missed L2 more)
+    static_assert(kTileBlocks % (kQThreads * 2) == 0, "a tile is whole units of every width");
+    fb.q_units = kTileBlocks / (kQThreads * BPT);
     const uint64_t n_tiles = static_cast<uint64_t>(fb.n_tensors) * fb.tiles;
-    fb.delay = fb.tiles + (n_tiles > static_cast<uint64_t>(res) ? static_cast<uint32_t>(res) : 0u);
-    fb.total = n_tiles + fb.delay;
-    fb.q_units = kTileBlocks / (kThreads * BPT);
-    const uint64_t grid = fb.total < static_cast<uint64_t>(res) ? fb.total : static_cast<uint64_t>(res);
+    const uint64_t grid = n_tiles < static_cast<uint64_t>(res) ? n_tiles : static_cast<uint64_t>(res);
+    // the amax warp may run one tensor and one and a half grids ahead of its CTA's quantize
+    // warps (two grids measured no faster and missed L2 more)
+    fb.window = fb.tiles + static_cast<uint32_t>(grid + grid / 2);
+    fb.n_sm = static_cast<uint32_t>(sm_count());
     return launch(kernel, dim3(static_cast<unsigned>(grid)), kThreads, s, fb);
 }
 

@@ -336,3 +336,25 @@ __device__ __forceinline__ bool mbar_test_parity(uint64_t* bar, uint32_t parity)
 }
 
 }  // namespace kvq
+
+namespace kvq {
+
+// Named barrier `id` among `threads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_volatile_smem(const uint32_t* p)
+{
+    uint32_t v;
+    asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_volatile_smem(uint32_t* p, uint32_t v)
+{
+    asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+
+}  // namespace kvq

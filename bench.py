@@ -103,6 +103,27 @@ def measured_launch_traffic(kind: str, shape: str):
     return float(k["dram_bytes_per_launch"])
 
 
+REL_MSE_BOUND = 2e-2  # relative MSE bound on N(0,1)-like inputs the method is held to
+
+
+def rel_mse(xs, ys) -> float:
+    """sum (y - x)^2 / sum x^2 in fp64 over pairs of bf16 tensors (the library's outputs
+    against its inputs, read back after the timed region)."""
+    num = den = 0.0
+    for x, y in zip(xs, ys):
+        xf, yf = x.reshape(-1).double(), y.reshape(-1).double()
+        num += float(((yf - xf) ** 2).sum())
+        den += float((xf ** 2).sum())
+    return num / den if den else 0.0
+
+
+def footprint(packed: int, scales: int, amax: int, elems: int, transient_bf16: int = 0) -> dict:
+    """Bytes of the quantized form against the bf16 it stands for."""
+    q = packed + scales + amax
+    return {"quantized_bytes": q, "bf16_bytes": 2 * elems, "ratio": 2 * elems / q if q else None,
+            "transient_bf16_bytes": transient_bf16}
+
+
 _CUDART = None
 
 
@@ -309,6 +330,23 @@ class Rollout:
     def tokens_per_step(self):
         return self.tokens * self.frames
 
+    def rel_mse(self):
+        """Layer 0's K and V over the whole rollout: the cache read back against the frames
+        appended into it."""
+        rows = self.frames * self.rpc
+        ys = self.kvq.kvq_dequantize_cache_batch(self.caches[0:2], 0, rows)
+        torch.cuda.synchronize()
+        xs = [self.x[:, t].reshape(-1) for t in range(2)]
+        return {"value": rel_mse(xs, ys), "bound": REL_MSE_BOUND,
+                "what": "layer 0 K and V, all frames, fp64: sum (y - x)^2 / sum x^2"}
+
+    def footprint(self):
+        """The full cache after the rollout (every layer's K and V) against its bf16 size, and
+        the bf16 buffers the per-layer reads reuse."""
+        pb, sb, ab = self.sizes
+        elems = 2 * self.layers * self.frames * self.chunk_elems
+        return footprint(pb, sb, ab, elems, 2 * self.yk.numel() * 2)
+
     def extra_rates(self, kind_ms):
         """Appended tokens/s of the append kernels, and prefix tokens/s of the reads
         (every layer, K and V, all heads of a token counted once)."""
@@ -380,6 +418,15 @@ class Layer:
         m = len(self.x)
         return self.p[:m] + self.s[:m] + self.a[:m] + self.y[:m]
 
+    def rel_mse(self):
+        m = len(self.x)
+        return {"value": rel_mse(self.x, self.y[:m]), "bound": REL_MSE_BOUND,
+                "what": f"{m} tensor(s), fp64: sum (y - x)^2 / sum x^2"}
+
+    def footprint(self):
+        m = len(self.x)
+        return footprint(m * self.n // 2, m * self.n // 16, 4 * m, m * self.n)
+
     def tokens_per_step(self):
         return self.tokens
 
@@ -442,6 +489,16 @@ class Cache:
 
     def d2h(self):
         return [self.p, self.s, self.a]
+
+    def rel_mse(self):
+        """The last layer's K and V (the pair the step dequantized last)."""
+        T = 2 * self.layers
+        return {"value": rel_mse([self.x[T - 2], self.x[T - 1]], [self.y[0], self.y[1]]), "bound": REL_MSE_BOUND,
+                "what": f"layer {self.layers - 1} K and V, fp64: sum (y - x)^2 / sum x^2"}
+
+    def footprint(self):
+        T = 2 * self.layers
+        return footprint(T * self.n // 2, T * self.n // 16, 4 * T, T * self.n, 2 * self.n * 2)
 
     def tokens_per_step(self):
         return self.tokens
@@ -582,6 +639,9 @@ class Rtn(Sweep):
 
     def d2h(self):
         return [self.p[0], self.s[0], self.y[0]]
+
+    def footprint(self):  # packed codes and one bf16 scale per 16 values
+        return footprint(self.n * self.bits // 8, self.n // 16 * 2, 0, self.n)
 
     def oracle_sample(self, orc, inputs, budget_s):
         m = min(self.tokens, 1 << 16)
@@ -1123,6 +1183,10 @@ def main():
 
     if hasattr(wl, "extra_rates"):
         line.update(wl.extra_rates({k: kind_ms[k] / args.steps for k in kinds}))
+    if hasattr(wl, "rel_mse"):
+        line["rel_mse"] = wl.rel_mse()
+    if hasattr(wl, "footprint"):
+        line["footprint"] = wl.footprint()
     if hasattr(wl, "check"):
         wl.check()
     if hasattr(wl, "unfused"):

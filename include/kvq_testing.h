@@ -21,6 +21,17 @@ extern "C" {
  */
 void kvq_testing_set_fused_wait(uint32_t extra_a_tiles, uint64_t wait_ns);
 
+/*
+ * kvq_testing_set_attention_wait -- for the current device: with wait_ns > 0, the MMA warp
+ *   of every later kvq_attention call first waits on an mbarrier that nothing arrives on,
+ *   and every data-path wait gives up after wait_ns nanoseconds. So the MMA warp issues
+ *   nothing, the other warps' waits give up in turn, the call lets whatever it issued
+ *   drain (that last wait keeps the library's 1 s bound), frees its tensor memory and
+ *   sets *status to 1. wait_ns == 0 restores normal operation. Call it while no
+ *   attention kernel runs on the device.
+ */
+void kvq_testing_set_attention_wait(uint64_t wait_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -93,6 +93,7 @@ def load() -> ctypes.CDLL:
     lib.kvq_device_status.argtypes, lib.kvq_device_status.restype = [I32], ctypes.c_int
     lib.kvq_testing_set_fused_wait.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
     lib.kvq_testing_set_fused_wait.restype = None
+    lib.kvq_testing_set_attention_wait.argtypes, lib.kvq_testing_set_attention_wait.restype = [ctypes.c_uint64], None
     _lib = lib
     return lib
 
@@ -141,6 +142,12 @@ def kvq_device_status(clear: bool = True) -> None:
     kernels gave up on the current device since the last clearing call (the word is
     cleared when ``clear``). Synchronize the streams of interest first."""
     _check(load().kvq_device_status(1 if clear else 0))
+
+
+def testing_set_attention_wait(wait_ns: int = 0) -> None:
+    """Test hook (kvq_testing.h): the bound of the attention kernel's data-path waits on
+    the current device (0 restores 1 s)."""
+    load().kvq_testing_set_attention_wait(int(wait_ns))
 
 
 def testing_set_fused_wait(extra_a_tiles: int, wait_ns: int = 0) -> None:

@@ -53,6 +53,7 @@
 #include "kvq.h"
 #include "kvq_common.h"
 #include "kvq_device.cuh"
+#include "kvq_testing.h"
 
 namespace kvq {
 namespace {
@@ -98,6 +99,13 @@ static_assert(kSoftmaxThreads == kProducerThreads && kProducerRegs <= 256 && kSo
                   kProducerRegs % 8 == 0 && kSoftmaxRegs >= 24 && 5 * 32 * kLaunchRegs <= 16384,
               "register split must balance");
 constexpr uint64_t kWaitNs = 1000000000ull;  // give up on an mbarrier after 1 s
+// The bound of the data-path waits: kWaitNs, shortened only by the test hook
+// kvq_testing_set_attention_wait. The final wait for the MMAs to drain before TMEM is
+// freed always keeps kWaitNs.
+__constant__ uint64_t c_wait_ns = kWaitNs;
+// Test hook: nonzero makes the MMA warp first wait on an mbarrier that nothing arrives on,
+// so the call's waits give up (after c_wait_ns) without any fault.
+__constant__ uint32_t c_stall_mma = 0;
 constexpr float kRescaleLog2 = 8.0f;          // rescale O when the row max grows by > 2^8
 constexpr int kMaxSplits = 64;
 constexpr int kCombineThreads = 256;  // 8 rows (warps) per CTA
@@ -107,6 +115,7 @@ constexpr uint64_t kPartialBytesPerRow = kD * 4 + 8;
 enum {
     kKFull0, kKFull1, kKEmpty0, kKEmpty1, kVFull0, kVFull1, kVEmpty0, kVEmpty1,
     kSFull0, kSFull1, kPFull0, kPFull1, kODone0, kODone1, kMmaDone,
+    kNever,  // never arrived on: the test hook's stalled wait
     kNumBars
 };
 
@@ -274,8 +283,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
-// Wait, for at most kWaitNs, for phase `parity` of an mbarrier; true when it completed.
-__device__ __forceinline__ bool wait_phase(uint32_t mbar, uint32_t parity)
+// Wait, for at most `limit` ns (the data-path bound by default), for phase `parity` of an
+// mbarrier; true when it completed.
+__device__ __forceinline__ bool wait_phase(uint32_t mbar, uint32_t parity, uint64_t limit = c_wait_ns)
 {
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
@@ -287,15 +297,15 @@ __device__ __forceinline__ bool wait_phase(uint32_t mbar, uint32_t parity)
                      : "memory");
         if (done)
             return true;
-        if (globaltimer_ns() - t0 > kWaitNs)
+        if (globaltimer_ns() - t0 > limit)
             return false;
     }
 }
 
 // The same wait, decided for the whole warp (tcgen05.ld/st need a converged warp).
-__device__ __forceinline__ bool warp_wait(uint32_t mbar, uint32_t parity)
+__device__ __forceinline__ bool warp_wait(uint32_t mbar, uint32_t parity, uint64_t limit = c_wait_ns)
 {
-    return __all_sync(0xFFFFFFFFu, wait_phase(mbar, parity));
+    return __all_sync(0xFFFFFFFFu, wait_phase(mbar, parity, limit));
 }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -712,6 +722,7 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
             mbar_init(bar(kODone0 + g), 1);
         }
         mbar_init(bar(kMmaDone), 1);
+        mbar_init(bar(kNever), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     // the query tiles -> shared memory (rows past n_q are zero; one tile with dual)
@@ -861,6 +872,8 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         const uint32_t sQ0 = base + G::kOffQ, sQ1 = dual ? sQ0 : base + G::kOffQ + kTileBytes;
         bool ok = true;
         const int steps = rank == 0 ? n_lead : 0;
+        if (c_stall_mma && steps > 0)
+            ok = warp_wait(bar(kNever), 0);  // gives up after c_wait_ns: nothing is issued
         if (steps > 0) {
             // S_g(0) for each slot: stream tile 0 for both, or with dual tiles 0 and 1
             for (int g = 0; ok && g < n_qt; ++g) {
@@ -911,7 +924,7 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         }
         if (rank == 0) {
             commit<PAIR>(bar(kMmaDone));  // completes once every MMA issued has
-            if (!warp_wait(bar(kMmaDone), 0))
+            if (!warp_wait(bar(kMmaDone), 0, kWaitNs))  // the drain keeps the full bound
                 ok = false;
         }
         if (!ok && lane == 0)
@@ -1449,3 +1462,11 @@ kvq_status kvq_attention_noalloc(const void* q, int32_t n_queries, int32_t heads
 }
 
 }  // extern "C"
+
+extern "C" void kvq_testing_set_attention_wait(uint64_t wait_ns)
+{
+    const uint64_t v = wait_ns ? wait_ns : kWaitNs;
+    const uint32_t stall = wait_ns ? 1u : 0u;
+    cudaMemcpyToSymbol(c_wait_ns, &v, sizeof(v));
+    cudaMemcpyToSymbol(c_stall_mma, &stall, sizeof(stall));
+}

@@ -220,3 +220,32 @@ def test_attention_argument_errors():
     c64 = kvq.KVCache(64, 16, 64)
     with pytest.raises(kvq.KvqError):  # head_dim 64 unsupported
         kvq.kvq_attention(torch.zeros((4, 2, 64), dtype=torch.bfloat16, device="cuda"), c64, c64, 4)
+
+
+@pytest.mark.parametrize("n_q,heads,n_tokens", [(100, 2, 700), (1100, 2, 900)])
+def test_wait_that_gives_up_sets_status_and_the_next_call_is_exact(orc, n_q, heads, n_tokens):
+    """With the test hook the MMA warp first waits on an mbarrier nothing arrives on and
+    every wait gives up after 1 ms: status is 1 and the binding's check raises
+    KVQ_ERR_TIMEOUT. The call drains and frees its tensor memory, which the next call on
+    the same stream shows: status 0 and the oracle's result. 100 queries run on single
+    CTAs, 1100 on CTA pairs plus a remainder."""
+    caches, ocs = _filled_caches(orc, heads, n_tokens, 64, "mse", 23)
+    q = inputs.normal((n_q, heads, D), 29, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        kvq.testing_set_attention_wait(1_000_000)
+        kvq.kvq_attention(q, caches[0], caches[1], n_tokens, status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 1
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.kvq_attention(q, caches[0], caches[1], n_tokens, check=True)
+        assert e.value.status == 6
+    finally:
+        kvq.testing_set_attention_wait(0)
+    status.zero_()
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_tokens, status=status, check=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kb = ocs[0].dequantize(0, n_tokens * heads)
+    vb = ocs[1].dequantize(0, n_tokens * heads)
+    _check_close(orc, out, bits(q), kb, vb, n_q, n_tokens, heads, D ** -0.5)

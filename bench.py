@@ -897,8 +897,9 @@ class Attention:
     def oracle_sample(self, orc, inputs, budget_s):
         """Layer 0: the oracle appends the cache (untimed), then dequantizes K and V and
         computes query rows' attention in fp64 (timed), doubling the rows per batch until
-        the time budget is spent; the bytes are the layer's algorithmic bytes scaled by
-        the share of query rows done."""
+        the time budget is spent. The bytes credited are the whole dequantization of K and
+        V (read 0.5625, write 2 B per element, as the timed region does it in full) plus
+        the layer's algorithmic attention bytes scaled by the share of query rows done."""
         caches = [orc.Cache(self.frames * self.rpc, self.rpc, self.D) for _ in range(2)]
         for f in range(self.frames):
             for t in range(2):
@@ -916,7 +917,9 @@ class Attention:
                 break
             m *= 2
         dt = time.perf_counter() - t0
-        return self.bytes_layer * rows / self.tokens, dt, f"layer 0, {rows} of {self.tokens} query rows"
+        deq_bytes = 2 * self.n_keys * self.heads * self.D * B_DEQUANT
+        return (deq_bytes + self.bytes_layer * rows / self.tokens, dt,
+                f"layer 0: K and V dequantized in full, then {rows} of {self.tokens} query rows")
 
 
 WORKLOADS = {c.name: c for c in (Rollout, Layer, Cache, Single, Sweep, RoundTrip, Rtn, Attention, Recent, Layout)}

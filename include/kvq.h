@@ -281,11 +281,13 @@ kvq_status kvq_attention_launches(int32_t n_queries, int32_t heads, int64_t n_ke
  *   Arguments, result and errors are those of kvq_attention, plus:
  *   - sizes whose key split needs more than 32 MiB (kvq_attention_workspace_bytes above
  *     32 MiB) return KVQ_ERR_CAPACITY with the needed size in kvq_last_error();
- *   - the first call on a device looks up the array's device address (once per device,
- *     that device current); make that first call before any stream capture;
+ *   - every call looks up the array's device address on the current device (a host-side
+ *     query that allocates nothing; the first one on a device may load the library's
+ *     device code, so make the first call before any stream capture);
  *   - every call on a GPU shares the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race on it and must be ordered by the caller. Nothing
- *     in it needs to start at zero.
+ *     in it needs to start at zero: a call whose *status stays 0 writes every partial it
+ *     reads; after a wait that gave up (*status 1) out may hold an earlier call's data.
  */
 kvq_status kvq_attention_noalloc(const void* q, int32_t n_queries, int32_t heads, const kvq_cache* k_cache,
                                  const kvq_cache* v_cache, int64_t n_keys, float softmax_scale, void* out,

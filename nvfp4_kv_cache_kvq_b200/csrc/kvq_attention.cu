@@ -47,7 +47,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 #include <type_traits>
 
 #include "kvq.h"
@@ -423,8 +422,10 @@ struct RawPiece {
 // gs = RN(amax / 2688). With MARK, without a division: Markstein's correction step (P.
 // Markstein, "Computation of elementary functions on the IBM RISC System/6000 processor",
 // IBM J. Res. Dev. 34(1), 1990) with y = RN(1/2688): q = RN(amax y), r = amax - 2688 q
-// (exact as one fma), RN(q + r y). Compared with the IEEE quotient for every positive
-// finite fp32 amax, it differs only below 2^-119, where the quotient is subnormal; a
+// (exact as one fma), RN(q + r y). It equals the IEEE quotient for every fp32 amax from
+// 2^-119 up (checked exhaustively over the five binades from 2^-119 to 2^-114, which hold
+// every amax whose quotient is subnormal from there on, amax below about 2^-114.6, and
+// on a sample of the rest); below 2^-119 it does not. A
 // single CTA takes MARK when every chunk amax its keys use is in [2^-119, FLT_MAX] (the
 // IEEE division, with its rare slow path, in the producer loop cost 13 % of a single
 // CTA's time per key tile).
@@ -1403,31 +1404,21 @@ namespace kvq {
 namespace {
 
 constexpr uint64_t kNoAllocScratchBytes = uint64_t{32} << 20;  // 32 MiB
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) uint8_t g_attention_scratch[kNoAllocScratchBytes];
 
-// Device address of g_attention_scratch on the current device, looked up once per device
-// with that device current (in host code the array's name is only a host-side stand-in).
+// Device address of g_attention_scratch on the current device (in host code the array's
+// name is only a host-side stand-in). It is looked up on every call, a host-side query
+// that allocates nothing: a cached address would outlive a context reset
+// (cudaDeviceReset) and point into the destroyed context. The first lookup on a device
+// may load this file's device code.
 kvq_status scratch_address(void** ptr)
 {
-    static std::mutex mu;
-    static void* addr[kMaxDevices] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_attention_scratch);
     if (e != cudaSuccess)
-        return launched(e, "kvq_attention_noalloc (current device)");
-    if (dev < 0 || dev >= kMaxDevices)
-        return fail(KVQ_ERR_UNSUPPORTED, "kvq_attention_noalloc: device %d beyond the %d supported", dev, kMaxDevices);
-    std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_attention_scratch);
-        if (e != cudaSuccess)
-            return launched(e, "kvq_attention_noalloc (scratch address)");
-        addr[dev] = p;
-    }
-    *ptr = addr[dev];
+        return launched(e, "kvq_attention_noalloc (scratch address)");
+    *ptr = p;
     return KVQ_OK;
 }
 
@@ -1455,8 +1446,9 @@ kvq_status kvq_attention_noalloc(const void* q, int32_t n_queries, int32_t heads
     if (need > 0 && (st = scratch_address(&scratch)) != KVQ_OK)
         return st;
     // the same call as kvq_attention with the recommended workspace: the same key split,
-    // hence the same result; every partial the combine reads is written first, so the
-    // scratch needs no clearing
+    // hence the same result; when *status stays 0 every partial the combine reads was
+    // written first by this call, so the scratch needs no clearing (after a wait that
+    // gave up, *status is 1 and out may hold partials an earlier call left in the scratch)
     return kvq_attention(q, n_queries, heads, k_cache, v_cache, n_keys, softmax_scale, out, scratch, need, status,
                          stream);
 }

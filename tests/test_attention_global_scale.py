@@ -84,8 +84,10 @@ def test_constants_and_threshold(lib):
     ulp = 2.0 ** (-12 - 23)
     assert abs(y - 1.0 / 2688.0) <= ulp / 2
     assert "2688.0f" in src
-    # every fp32 amax in the 4 binades from the threshold up: the IEEE quotient
-    assert lib.mismatches(_bits(lo), _bits(lo * 16.0), y, 2688.0) == 0
+    # every fp32 amax in the 5 binades from the threshold up, through the whole range where
+    # the quotient amax / 2688 is subnormal (amax below about 2^-114.6) and into normal
+    # quotients: the IEEE quotient
+    assert lib.mismatches(_bits(lo), _bits(lo * 32.0), y, 2688.0) == 0
     # just below it the step is not exact (the quotient is subnormal): the kernel divides
     assert lib.mismatches(_bits(lo / 4.0), _bits(lo), y, 2688.0) > 0
 

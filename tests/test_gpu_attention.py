@@ -187,7 +187,8 @@ def test_attention_launch_count():
 def test_attention_rollout_shape_sampled(orc):
     """The rollout's attention at full size -- one frame of 1560 queries x 12 heads over a
     60-frame cache (93,600 keys) appended frame by frame with the mse rule -- checked on a
-    sample of query rows (the oracle computes those rows only)."""
+    sample of query rows of the pair part and on every row of the 24-row remainder that
+    runs on single CTAs (the oracle computes those rows only)."""
     heads, tpc, frames = 12, inputs.TOKENS_PER_FRAME, 60
     rpc = tpc * heads
     caches = [kvq.KVCache(frames * rpc, rpc, D) for _ in range(2)]
@@ -203,7 +204,7 @@ def test_attention_rollout_shape_sampled(orc):
     out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    rows = torch.tensor([0, 1, 127, 128, 777, 1400, 1535, 1559])
+    rows = torch.tensor([0, 1, 127, 128, 777, 1400, 1535] + list(range(1536, 1560)))
     kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
     _check_close(orc, out[rows.cuda()], bits(q[rows.cuda()]), kb, vb, len(rows), n_keys, heads, D ** -0.5)
 
@@ -244,6 +245,27 @@ def test_wait_that_gives_up_sets_status_and_the_next_call_is_exact(orc, n_q, hea
         kvq.testing_set_attention_wait(0)
     status.zero_()
     out = kvq.kvq_attention(q, caches[0], caches[1], n_tokens, status=status, check=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kb = ocs[0].dequantize(0, n_tokens * heads)
+    vb = ocs[1].dequantize(0, n_tokens * heads)
+    _check_close(orc, out, bits(q), kb, vb, n_q, n_tokens, heads, D ** -0.5)
+
+
+@pytest.mark.parametrize("fraction", [0.5, 0.1])
+def test_smaller_workspace_than_recommended(orc, fraction):
+    """A workspace smaller than recommended (but not empty) makes the launch plan shrink:
+    fewer key splits for the part with the most partials, then no dual mode, offsets
+    recomputed. 600 queries x 4 heads run a pair part and a remainder part; the result
+    stays within the oracle's bound."""
+    n_q, heads, n_tokens = 600, 4, 5000
+    caches, ocs = _filled_caches(orc, heads, n_tokens, 500, "mse", 31)
+    q = inputs.normal((n_q, heads, D), 37, "cuda")
+    need = kvq.kvq_attention_workspace_bytes(n_q, heads, n_tokens)
+    assert need > 0 and kvq.kvq_attention_launches(n_q, heads, n_tokens) >= 3
+    ws = torch.empty(int(need * fraction) // 256 * 256, dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_tokens, workspace=ws, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     kb = ocs[0].dequantize(0, n_tokens * heads)

@@ -1165,8 +1165,15 @@ def main():
                     "roundtrip": B_AMAX + B_QUANT + 2.0, "rtn_quantize": 2.0 + args.bits / 8 + 2.0 / 16,
                     "rtn_dequantize": 2.0 + args.bits / 8 + 2.0 / 16,
                     "to_blocked": 2.0, "from_blocked": 2.0}.get(dom)  # layout: per scale byte
-        # the RTN codecs' traffic depends on the bit width: their entries carry it
-        tb = measured_traffic(f"{dom}_int{args.bits}" if dom.startswith("rtn_") else dom) if per_elem else None
+        # the RTN codecs' traffic depends on the bit width: their entries carry it; a
+        # quantize with its own amax runs in one launch (plus the slot fill) up to 2^21
+        # blocks per tensor, else as two passes
+        key = dom
+        if dom.startswith("rtn_"):
+            key = f"{dom}_int{args.bits}"
+        elif dom == "quantize" and kind_launch[dom] == 2 * sum(1 for s_ in segs if s_.kind == dom):
+            key = "quantize_one_launch"
+        tb = measured_traffic(key) if per_elem else None
         elems_per_launch = kind_bytes[dom] / per_elem / kind_launch[dom] if per_elem else None
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)",

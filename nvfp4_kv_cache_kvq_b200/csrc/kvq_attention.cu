@@ -667,10 +667,10 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
     const int unit = PAIR ? blockIdx.x >> 1 : blockIdx.x, split = blockIdx.y, h = blockIdx.z;
     const int t_begin = static_cast<int>(static_cast<int64_t>(split) * a.key_tiles / gridDim.y);
     const int t_end = static_cast<int>(static_cast<int64_t>(split + 1) * a.key_tiles / gridDim.y);
-    const int n_tiles = t_end - t_begin;
     const int64_t u0 = static_cast<int64_t>(unit) * G::kRowsPerUnit;   // first row of the unit
     const int64_t q0 = u0 + rank * kBM;                                // this CTA's first row
     constexpr int kSlotRows = G::kCtas * kBM;                          // rows between slots
+    const int n_tiles = t_end - t_begin;
     // dual: both slots hold query tile 0; slot 0 takes the first n_lead key tiles of the
     // range, slot 1 the rest, and each writes its own partial result (2 split + slot)
     constexpr bool dual = DUAL;
@@ -946,27 +946,31 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
         auto produce = [&](auto mark_tag) {
             constexpr bool MARK = decltype(mark_tag)::value;
             const int p = tid - kSoftmaxThreads;
-            auto key0_of = [&](int s) { return static_cast<int64_t>(key_tile(s)) * kBN; };
             const int k_q = p & 3, v_q = p % G::kVQuarters;
             auto k_row = [&](int i) { return (p + kProducerThreads * i) >> 2; };
             auto v_row = [&](int i) { return (p + kProducerThreads * i) / G::kVQuarters; };
-            auto k_key = [&](int j, int i) { return key0_of(j) + rank * (kBN - G::kKRows) + k_row(i); };
-            auto v_key = [&](int j, int i) { return key0_of(j) + v_row(i); };
+            // the first key of the K and V tile loaded last: each load_x(j) is followed by
+            // put_x(j) before the next load_x
+            int64_t k_key0 = 0, v_key0 = 0;
+            auto k_key = [&](int i) { return k_key0 + rank * (kBN - G::kKRows) + k_row(i); };
+            auto v_key = [&](int i) { return v_key0 + v_row(i); };
             RawPiece rk[G::kKPieces], rv[G::kVPieces];
             auto load_k = [&](int j) {
+                k_key0 = static_cast<int64_t>(key_tile(j)) * kBN;
     #pragma unroll
                 for (int i = 0; i < G::kKPieces; ++i)
-                    load_piece(a.kp, a.ks, a.ka, a, h, k_key(j, i), k_q, rk[i]);
+                    load_piece(a.kp, a.ks, a.ka, a, h, k_key(i), k_q, rk[i]);
             };
             auto load_v = [&](int j) {
+                v_key0 = static_cast<int64_t>(key_tile(j)) * kBN;
     #pragma unroll
                 for (int i = 0; i < G::kVPieces; ++i)
-                    load_piece(a.vp, a.vs, a.va, a, h, v_key(j, i), v_q + static_cast<int>(rank) * G::kVQuarters, rv[i]);
+                    load_piece(a.vp, a.vs, a.va, a, h, v_key(i), v_q + static_cast<int>(rank) * G::kVQuarters, rv[i]);
             };
             auto put_k = [&](int j) {
     #pragma unroll
                 for (int i = 0; i < G::kKPieces; ++i)
-                    store_piece<MARK>(rk[i], k_key(j, i) < a.n_kv, k_row(i), k_q >> 1, (k_q & 1) * 4, G::kKRows, (k_q & 2) != 0,
+                    store_piece<MARK>(rk[i], k_key(i) < a.n_kv, k_row(i), k_q >> 1, (k_q & 1) * 4, G::kKRows, (k_q & 2) != 0,
                                 sK(j));
                 fence_async_smem();
                 __syncwarp();
@@ -976,7 +980,7 @@ __global__ void __maxnreg__(kLaunchRegs) attention_kernel(const AttnArgs a)
             auto put_v = [&](int j) {
     #pragma unroll
                 for (int i = 0; i < G::kVPieces; ++i)
-                    store_piece<MARK>(rv[i], v_key(j, i) < a.n_kv, v_row(i), v_q >> 1, (v_q & 1) * 4, kBN, (v_q & 2) != 0,
+                    store_piece<MARK>(rv[i], v_key(i) < a.n_kv, v_row(i), v_q >> 1, (v_q & 1) * 4, kBN, (v_q & 2) != 0,
                                 sV(j));
                 fence_async_smem();
                 __syncwarp();

@@ -110,6 +110,27 @@ def test_attention_matches_oracle(orc, n_q, heads, n_keys, tokens_per_chunk, rul
     _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, scale)
 
 
+@pytest.mark.parametrize("n_q,heads,n_keys,tokens_per_chunk,rule", [
+    # one pair unit and a 24-row dual part: the pair launch's 61 key ranges hold 4 or 5
+    # tiles, the dual CTAs' 50 ranges 6 or 7 (slots of 3 and 3, or 4 and 3)
+    (536, 1, 301 * 128 - 5, 1000, "mse"),
+    # two pair units per head over 17 key ranges of 5 or 6 tiles; a 100-row dual part
+    # over 50 ranges of 2 tiles (one per slot)
+    (1124, 2, 100 * 128, 128, "static_6"),
+])
+def test_pairs_then_dual_with_ragged_key_ranges(orc, n_q, heads, n_keys, tokens_per_chunk, rule):
+    """A pair part followed by a dual part, both over key ranges of unequal length."""
+    assert kvq.kvq_attention_launches(n_q, heads, n_keys) == 4
+    caches, ocs = _filled_caches(orc, heads, n_keys, tokens_per_chunk, rule, 700)
+    q = inputs.normal((n_q, heads, D), 13, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = kvq.kvq_attention(q, caches[0], caches[1], n_keys, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kb, vb = ocs[0].dequantize(0, n_keys * heads), ocs[1].dequantize(0, n_keys * heads)
+    _check_close(orc, out, bits(q), kb, vb, n_q, n_keys, heads, D ** -0.5)
+
+
 def test_attention_many_key_splits(orc):
     """One query tile of one head over 64 key tiles: the split heuristic spreads the keys
     over the most units (up to 64), so the combine merges many partials."""

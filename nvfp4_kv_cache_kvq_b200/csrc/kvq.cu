@@ -450,7 +450,7 @@ constexpr unsigned kDeviceErrWaitTimeout = 1u;
 //   amax is complete, meeting among themselves at a named barrier per tile (amax
 //   broadcast, scale tables).
 // The amax warp runs ahead of its own CTA's quantize warps by at most `window` tiles (one
-// tensor and one and a half grids): far enough that a tensor's amax is mostly complete
+// tensor and two grids): far enough that a tensor's amax is mostly complete
 // before its quantize tiles ask for it, close enough that the tiles in between are still
 // in L2 when they are quantized (a global throttle, an amax warp waiting for tensor t - L
 // to be quantized everywhere, measured slower and missed L2 on most re-reads). A tensor
@@ -513,14 +513,18 @@ __device__ __forceinline__ uint32_t await_amax(const FusedBatch& B, uint32_t t)
     uint32_t* slot = slot_of(B, t);
     uint32_t v = ld_relaxed_u32(slot);
     if (!slot_complete(v, B.expect_a)) {
+        // polls back off from 64 to 512 ns: the slot is one word that every CTA of the
+        // tensor reads and its amax tiles fold into (measured 3 % faster than 64 ns polls)
         const uint64_t t0 = globaltimer_ns();
+        uint32_t ns = 64;
         while (!slot_complete(v = ld_relaxed_u32(slot), B.expect_a)) {
             if (globaltimer_ns() - t0 > B.wait_ns) {
                 st_relaxed_u32(slot, kNaNBits);
                 atomicOr(&g_device_error, kDeviceErrWaitTimeout);
                 return kNaNBits;
             }
-            __nanosleep(64);
+            __nanosleep(ns);
+            ns = ns < 512u ? 2 * ns : ns;
         }
     }
     if ((v & 0xFFFF0000u) == kNaNBits)
@@ -807,9 +811,10 @@ cudaError_t launch_fused(FusedBatch& fb, cudaStream_t s)
     fb.q_units = kTileBlocks / (kQThreads * BPT);
     const uint64_t n_tiles = static_cast<uint64_t>(fb.n_tensors) * fb.tiles;
     const uint64_t grid = n_tiles < static_cast<uint64_t>(res) ? n_tiles : static_cast<uint64_t>(res);
-    // the amax warp may run one tensor and one and a half grids ahead of its CTA's quantize
-    // warps (two grids measured no faster and missed L2 more)
-    fb.window = fb.tiles + static_cast<uint32_t>(grid + grid / 2);
+    // the amax warp may run one tensor and two grids ahead of its CTA's quantize warps
+    // (measured on the rollout's appends: 5 % faster than one and a half grids, three grids
+    // slower)
+    fb.window = fb.tiles + static_cast<uint32_t>(2 * grid);
     fb.n_sm = static_cast<uint32_t>(sm_count());
     return launch(kernel, dim3(static_cast<unsigned>(grid)), kThreads, s, fb);
 }

@@ -323,11 +323,14 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                  : "memory");
 }
 
-__device__ __forceinline__ bool mbar_test_parity(uint64_t* bar, uint32_t parity)
+// Phase `parity` of the mbarrier is complete. try_wait lets the hardware suspend the
+// thread for a while before it answers false, so a caller's wait loop issues few
+// instructions.
+__device__ __forceinline__ bool mbar_try_parity(uint64_t* bar, uint32_t parity)
 {
     uint32_t done;
     asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
                  "selp.u32 %0, 1, 0, p;\n\t}"
                  : "=r"(done)
                  : "r"(smem_addr(bar)), "r"(parity)

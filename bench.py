@@ -110,10 +110,13 @@ def rel_mse(xs, ys) -> float:
     """sum (y - x)^2 / sum x^2 in fp64 over pairs of bf16 tensors (the library's outputs
     against its inputs, read back after the timed region)."""
     num = den = 0.0
+    step = 1 << 26  # elements per fp64 pass (512 MB per temporary)
     for x, y in zip(xs, ys):
-        xf, yf = x.reshape(-1).double(), y.reshape(-1).double()
-        num += float(((yf - xf) ** 2).sum())
-        den += float((xf ** 2).sum())
+        xr, yr = x.reshape(-1), y.reshape(-1)
+        for i in range(0, xr.numel(), step):
+            xf, yf = xr[i:i + step].double(), yr[i:i + step].double()
+            num += float(((yf - xf) ** 2).sum())
+            den += float((xf ** 2).sum())
     return num / den if den else 0.0
 
 

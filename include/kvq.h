@@ -98,8 +98,9 @@ typedef enum {
  *            copy of *amax_in). At least one of amax_in / amax_out must be non-NULL.
  *   packed   device, uint8[n_elems / 2], 8-byte aligned. Written.
  *   scales   device, uint8[n_elems / 16] (e4m3 codes, one per block, same order). Written.
- * When the amax is computed, amax pass and quantization run in one launch for tensors of
- * up to about 2^25 blocks (larger ones take two): the tiles of the amax pass fold their
+ * When the amax is computed for a batch of two or more tensors of up to 2^21 blocks (64
+ * MiB of bf16) each (kvq_quantize_batch, kvq_append_batch), amax pass and quantization
+ * run in one launch (otherwise in two): the tiles of the amax pass fold their
  * maxima into *amax_out, and the quantize tiles of the same launch wait for it there, so
  * the slot holds intermediate values until the stream reaches the end of the call. Such
  * a wait is bounded (2 s); if it gives up, the tensor's outputs are left unwritten,
@@ -141,9 +142,10 @@ kvq_status kvq_quantize_batch(const void* const* xs, int32_t n_tensors, int64_t 
  * kvq_quantize_launches -- host only: the number of kernels kvq_quantize_batch (and
  *   kvq_append_batch, kvq_quantize_dequantize) launches for n_tensors tensors of n_elems
  *   elements: per group of KVQ_MAX_BATCH tensors, 1 when the amax is given (amax_given
- *   != 0), else 2 (a slot clear and the one-launch amax + quantize) or 3 (clear, amax
- *   pass, quantize) for tensors too large for one launch. For 16-byte-aligned packed
- *   buffers; writes *launches (0 for empty tensors).
+ *   != 0), else 2 (a slot clear and the one-launch amax + quantize, for groups of two or
+ *   more tensors of up to 2^21 blocks each) or 3 (clear, amax pass, quantize: a single
+ *   tensor, or larger tensors). For 16-byte-aligned packed buffers; writes *launches (0
+ *   for empty tensors).
  */
 kvq_status kvq_quantize_launches(int32_t n_tensors, int64_t n_elems, int32_t head_dim, int32_t amax_given,
                                  int32_t* launches);

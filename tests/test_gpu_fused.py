@@ -1,12 +1,13 @@
-"""The one-launch amax + quantize path (fused_quantize_kernel) against the oracle, around
-every switch of its launch plan, and its bounded wait made to give up on purpose.
+"""The one-launch amax + quantize path (fused_quantize_kernel, taken by batches of two or
+more tensors) against the oracle, around every switch of its launch plan, and its bounded
+wait made to give up on purpose.
 
 Amax and quantize tiles of 896 blocks (7 quantize warps x 2 units x 2 blocks): ragged
-last tiles, one and several tiles, one and several tensors, jobs within one wave of CTAs
+last tiles, one and several tiles, two and three tensors, jobs within one wave of CTAs
 and jobs over several waves (the amax warps then run ahead of the quantize warps, up to
-a tensor and two grids), the largest tensor the launch takes (64 MiB of bf16) and the
-next size, which takes the separate amax pass; two blocks per thread and one (packed /
-scales alignment); the three output modes."""
+a tensor and one and a half grids), the largest tensors the launch takes (64 MiB of bf16
+each) and the next size, which takes the separate amax pass, as does a single tensor; two
+blocks per thread and one (packed / scales alignment)."""
 import numpy as np
 import pytest
 import torch
@@ -43,7 +44,7 @@ def _check_batch(orc, xs, rule, offset_bytes=0):
 
 
 @pytest.mark.parametrize("blocks", [8, 888, 896, 904, 65536 + 8])
-@pytest.mark.parametrize("n_tensors", [1, 3])
+@pytest.mark.parametrize("n_tensors", [2, 3])
 def test_plan_switch_tile_size(orc, blocks, n_tensors):
     rows = -(-blocks // 8)
     xs = [_x(rows, 100 * n_tensors + i) for i in range(n_tensors)]
@@ -72,47 +73,36 @@ def test_several_waves(orc):
         check_sampled(orc, xs[i], p[i], s[i], float(a[i].cpu()[0]), None, "mse", seed=i)
 
 
-def test_largest_one_launch_tensor_and_the_two_pass_above(orc):
+def test_largest_one_launch_tensors_and_the_two_pass_above(orc):
     """2^21 blocks (64 MiB of bf16) is the largest tensor of the one-launch path; one row
-    more takes the separate amax pass."""
+    more takes the separate amax pass. A single tensor always does."""
+    assert kvq.kvq_quantize_launches(1, 1024 * 128) == 3
+    assert kvq.kvq_quantize_launches(65, 1024 * 128) == 2 + 3  # a group of 64, then one
     for rows in (262_144, 262_145):
-        assert kvq.kvq_quantize_launches(1, rows * 128) == (2 if rows == 262_144 else 3)
-        x = _x(rows, 9)
-        p, s, a = kvq.kvq_quantize(x, 128, "mse")
+        assert kvq.kvq_quantize_launches(2, rows * 128) == (2 if rows == 262_144 else 3)
+        xs = [_x(rows, 9), _x(rows, 10)]
+        p, s, a = kvq.kvq_quantize_batch(xs, 128, "mse")
         torch.cuda.synchronize()
         kvq.kvq_device_status()
-        check_sampled(orc, x, p, s, float(a.cpu()[0]), None, "mse")
-        del x, p, s, a
-
-
-def test_round_trip_modes_in_one_launch(orc):
-    x = _x(20000, 11)
-    y, p, s, a = kvq.kvq_quantize_dequantize(x, 128, "mse")
-    y2, _, _, a2 = kvq.kvq_quantize_dequantize(x, 128, "mse", codes=False)
-    torch.cuda.synchronize()
-    pe, se, ae = orc.quantize(bits(x), 128, "mse")
-    assert float(a.cpu()[0]) == ae and float(a2.cpu()[0]) == ae
-    assert_same(p.cpu().numpy(), pe, "packed")
-    assert_same(s.cpu().numpy(), se, "scales")
-    want = orc.dequantize(pe, se, ae, 128)
-    assert_same(bits(y), want, "y")
-    assert_same(bits(y2), want, "y codes=False")
+        for i in range(2):
+            check_sampled(orc, xs[i], p[i], s[i], float(a[i].cpu()[0]), None, "mse", seed=i)
+        del xs, p, s, a
 
 
 def test_bounded_wait_gives_up_and_the_next_call_is_correct(orc):
     """With the test hook, every quantize tile waits for one amax tile more than exist;
     the wait gives up after 2 ms: nothing is written, the amax is NaN, and
-    kvq_device_status reports the timeout. Then the same call without the hook is exact,
-    on the same stream, in the same process."""
-    x = _x(4096, 12)
-    n = x.numel()
-    packed = torch.full((n // 2,), 0xA5, dtype=torch.uint8, device="cuda")
-    scales = torch.full((n // 16,), 0x5A, dtype=torch.uint8, device="cuda")
-    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    kvq_device_status reports the timeout. Then the same calls without the hook are
+    exact, on the same stream, in the same process."""
+    xs = [_x(4096, 12), _x(4096, 13)]
+    n = xs[0].numel()
+    packed = [torch.full((n // 2,), 0xA5, dtype=torch.uint8, device="cuda") for _ in xs]
+    scales = [torch.full((n // 16,), 0x5A, dtype=torch.uint8, device="cuda") for _ in xs]
+    amax = [torch.zeros(1, dtype=torch.float32, device="cuda") for _ in xs]
     kvq.kvq_device_status()  # clear
     try:
         kvq.testing_set_fused_wait(1, 2_000_000)
-        kvq.kvq_quantize(x, 128, "mse", amax_out=amax, packed=packed, scales=scales)
+        kvq.kvq_quantize_batch(xs, 128, "mse", amax_out=amax, packed=packed, scales=scales)
         torch.cuda.synchronize()
     finally:
         kvq.testing_set_fused_wait(0, 0)
@@ -120,26 +110,28 @@ def test_bounded_wait_gives_up_and_the_next_call_is_correct(orc):
         kvq.kvq_device_status()
     assert e.value.status == 6
     kvq.kvq_device_status()  # cleared by the call above
-    assert torch.isnan(amax).all()
-    assert bool((packed == 0xA5).all()) and bool((scales == 0x5A).all())
+    for i in range(2):
+        assert torch.isnan(amax[i]).all()
+        assert bool((packed[i] == 0xA5).all()) and bool((scales[i] == 0x5A).all())
     # an append under the hook times out the same way
-    cache = kvq.allocate_caches(1, 1, 4096, 128, 4096, "cuda")[0]
+    caches = kvq.allocate_caches(1, 1, 4096, 128, 4096, "cuda")
     try:
         kvq.testing_set_fused_wait(1, 2_000_000)
-        kvq.kvq_append(cache, 0, x, "mse")
+        kvq.kvq_append_batch(caches, [0, 0], xs, "mse")
         torch.cuda.synchronize()
     finally:
         kvq.testing_set_fused_wait(0, 0)
     with pytest.raises(kvq.KvqError):
         kvq.kvq_device_status()
     # normal operation resumes
-    kvq.kvq_quantize(x, 128, "mse", amax_out=amax, packed=packed, scales=scales)
-    kvq.kvq_append(cache, 0, x, "mse")
+    kvq.kvq_quantize_batch(xs, 128, "mse", amax_out=amax, packed=packed, scales=scales)
+    kvq.kvq_append_batch(caches, [0, 0], xs, "mse")
     torch.cuda.synchronize()
     kvq.kvq_device_status()
-    pe, se, ae = orc.quantize(bits(x), 128, "mse")
-    assert float(amax.cpu()[0]) == ae and float(cache.amax.cpu()[0]) == ae
-    assert_same(packed.cpu().numpy(), pe, "packed")
-    assert_same(scales.cpu().numpy(), se, "scales")
-    assert_same(cache.packed.cpu().numpy(), pe, "cache packed")
-    assert np.array_equal(cache.scales.cpu().numpy(), se)
+    for i in range(2):
+        pe, se, ae = orc.quantize(bits(xs[i]), 128, "mse")
+        assert float(amax[i].cpu()[0]) == ae and float(caches[i].amax.cpu()[0]) == ae
+        assert_same(packed[i].cpu().numpy(), pe, "packed")
+        assert_same(scales[i].cpu().numpy(), se, "scales")
+        assert_same(caches[i].packed.cpu().numpy(), pe, "cache packed")
+        assert np.array_equal(caches[i].scales.cpu().numpy(), se)

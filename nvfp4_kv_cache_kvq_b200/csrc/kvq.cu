@@ -847,8 +847,8 @@ bool plan_fused(uint64_t n_blocks, int n, FusedBatch& fb)
 
 // Quantize a batch of equally sized tensors whose amax slots are given. When
 // compute_amax, the amax is reduced into the slots first: in the same launch
-// (fused_quantize_kernel) for tensors of up to kFusedMaxBlocks blocks, else by
-// amax_kernel before quantize_kernel.
+// (fused_quantize_kernel) for two or more tensors of up to kFusedMaxBlocks blocks
+// (codes only), else by amax_kernel before quantize_kernel.
 kvq_status run_quantize(const QuantBatch& qb, int n, bool compute_amax, kvq_scale_rule rule, cudaStream_t s,
                         int mode = kCodes)
 {

@@ -62,6 +62,25 @@ def test_host_only_calls():
     assert e.value.status == 1
 
 
+def test_quantize_launch_plan():
+    """The launch plan kvq_quantize_launches reports (host only): a batch of two or more
+    tensors of up to 2^21 blocks takes the slot fill and one amax + quantize launch; a
+    single tensor, or a larger one, the fill, the amax pass and the quantize pass; a given
+    amax, the quantize pass alone; each group of 64 tensors is planned on its own."""
+    big = (1 << 21) * 16  # elements of the largest one-launch tensor
+    assert kvq.kvq_quantize_launches(1, 4096 * 128) == 3
+    assert kvq.kvq_quantize_launches(2, 4096 * 128) == 2
+    assert kvq.kvq_quantize_launches(60, 1560 * 12 * 128) == 2
+    assert kvq.kvq_quantize_launches(2, big) == 2
+    assert kvq.kvq_quantize_launches(2, big + 128) == 3
+    assert kvq.kvq_quantize_launches(64, 128) == 2
+    assert kvq.kvq_quantize_launches(65, 128) == 2 + 3  # 64, then a single tensor
+    assert kvq.kvq_quantize_launches(66, 128) == 2 + 2
+    assert kvq.kvq_quantize_launches(130, 128, amax_given=True) == 3
+    assert kvq.kvq_quantize_launches(0, 128) == 0
+    assert kvq.kvq_quantize_launches(2, 0) == 0
+
+
 def _fake(addr):
     return ctypes.c_void_p(addr)
 

@@ -106,11 +106,10 @@ def measured_launch_traffic(kind: str, shape: str):
 REL_MSE_BOUND = 2e-2  # relative MSE bound on N(0,1)-like inputs the method is held to
 
 
-def rel_mse(xs, ys) -> float:
+def rel_mse(xs, ys, step: int = 1 << 26) -> float:
     """sum (y - x)^2 / sum x^2 in fp64 over pairs of bf16 tensors (the library's outputs
     against its inputs, read back after the timed region)."""
-    num = den = 0.0
-    step = 1 << 26  # elements per fp64 pass (512 MB per temporary)
+    num = den = 0.0  # summed over passes of `step` elements (fp64 temporaries of 8 step bytes)
     for x, y in zip(xs, ys):
         xr, yr = x.reshape(-1), y.reshape(-1)
         for i in range(0, xr.numel(), step):

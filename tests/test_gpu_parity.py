@@ -74,6 +74,25 @@ def test_layer_kv(orc, rule):
         check_full(orc, inputs.layer_kv(kv, device="cuda"), rule, 128)
 
 
+@pytest.mark.parametrize("rule", RULES)
+def test_layer_kv_batched_as_the_benchmark_runs_it(orc, rule):
+    """The layer workload in the benchmark's launch configuration: K and V in one
+    kvq_quantize_batch (the amax and the codes in one launch) and one kvq_dequantize_batch,
+    whole tensors against the oracle."""
+    xs = [inputs.layer_kv(kv, device="cuda") for kv in (0, 1)]
+    assert kvq.kvq_quantize_launches(2, xs[0].numel()) == 2
+    p, s, a = kvq.kvq_quantize_batch(xs, 128, rule)
+    ys = kvq.kvq_dequantize_batch(p, s, a, 128)
+    torch.cuda.synchronize()
+    kvq.kvq_device_status()
+    for i, x in enumerate(xs):
+        pe, se, ae = orc.quantize(bits(x), 128, rule)
+        assert float(a[i][0]) == ae
+        assert_same(s[i].cpu().numpy(), se, f"scales t{i}")
+        assert_same(p[i].cpu().numpy(), pe, f"packed t{i}")
+        assert_same(bits(ys[i]), orc.dequantize(pe, se, ae, 128), f"dequant t{i}")
+
+
 def _all_bf16(lo: float, hi: float) -> np.ndarray:
     """Every finite bf16 bit pattern with lo <= value <= hi (both signs if lo < 0)."""
     u = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)

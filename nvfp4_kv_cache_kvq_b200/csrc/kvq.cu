@@ -453,11 +453,13 @@ constexpr unsigned kDeviceErrWaitTimeout = 1u;
 // tensor and one and a half grids): far enough that a tensor's amax is mostly complete
 // before its quantize tiles ask for it, close enough that the tiles in between are still
 // in L2 when they are quantized (a global throttle, an amax warp waiting for tensor t - L
-// to be quantized everywhere, measured slower and missed L2 on most re-reads). A tensor
-// the quantize warps wait for has all its amax tiles within the reach of the CTAs that
-// own them: each of those CTAs' quantize warps is at or past that tensor, and the window
-// covers a whole tensor beyond it. So no wait depends on itself. The quantize warps share
-// nothing with the amax warp but the position they publish.
+// to be quantized everywhere, measured slower and missed L2 on most re-reads). Progress,
+// by induction over the tensors: let t be the first tensor whose amax is incomplete. The
+// quantize warps of a CTA owning one of t's amax tiles do not wait on earlier tensors, so
+// they reach a tile of tensor t or later (position >= t's first tile) or finish; the
+// window, at least one tensor, then reaches every tile of t, so the CTA's amax warp folds
+// its tiles of t and t completes. With every CTA resident, each wait ends. The quantize
+// warps share nothing with the amax warp but the position they publish.
 //
 // The synchronisation lives in the caller's amax slot, so the launch needs no memory of
 // its own. fill_kernel sets the slot to kSlotBase before the launch; then

@@ -81,3 +81,33 @@ def test_binding_signature_matches_header(name):
         assert fn.restype is ctypes.c_char_p
     else:
         assert fn.restype in (ctypes.c_int, ctypes.c_int32)
+
+
+def _structs():
+    """typedef struct { fields } name; -> {name: [(field, 'pointer' or ctypes type)]}."""
+    out = {}
+    src = open(HEADERS[0]).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    for m in re.finditer(r"typedef\s+struct\s*\{([^}]*)\}\s*(\w+)\s*;", src):
+        fields = []
+        for decl in m.group(1).split(";"):
+            decl = decl.strip()
+            if not decl:
+                continue
+            name = re.search(r"(\w+)$", decl).group(1)
+            fields.append((name, _kind(decl)))
+        out[m.group(2)] = fields
+    return out
+
+
+@pytest.mark.parametrize("c_name,py_struct", [("kvq_cache", "_Cache"), ("kvq_recent_cache", "_RecentCache")])
+def test_binding_structs_match_header(c_name, py_struct):
+    """Field order, kind and width of the cache views the binding passes by pointer."""
+    want = _structs()[c_name]
+    got = getattr(kvq, py_struct)._fields_
+    assert [f for f, _ in got] == [f for f, _ in want]
+    for (f, t), (_, k) in zip(got, want):
+        if k == "pointer":
+            assert _is_pointer_ctype(t), (c_name, f)
+        else:
+            assert not _is_pointer_ctype(t) and ctypes.sizeof(t) == ctypes.sizeof(k), (c_name, f)

@@ -101,16 +101,19 @@ def _random_blocks(rng, n):
         if kind == 3 and k % 2:
             amax_t = amax_b * 448.0  # gs = amax_b / 6: every product val * S is exact
         else:
-            amax_t = amax_b * float(rng.choice([1.0, 1.0, 2.5, 37.0, 1e3]))
+            # up to 1e3: normal e4m3 scales; 1e5 and 3e6: subnormal e4m3 scales and scales
+            # that round to zero (448 * amax_b / amax_t below 2^-6 and 2^-10)
+            amax_t = amax_b * float(rng.choice([1.0, 1.0, 2.5, 37.0, 1e3, 1e5, 3e6]))
         out.append((x, float(np.float32(amax_t))))
     return out
 
 
 def test_oracle_equals_exact_restatement_bit_for_bit(orc):
     rng = np.random.default_rng(2026)
-    blocks = _random_blocks(rng, 400)
-    assert len(blocks) > 350
+    blocks = _random_blocks(rng, 600)
+    assert len(blocks) > 500
     chose4 = 0
+    subnormal_scales = 0
     for x, amax_f in blocks:
         amax_t = Fraction(amax_f)
         bits = [int(b) for b in x]
@@ -119,8 +122,10 @@ def test_oracle_equals_exact_restatement_bit_for_bit(orc):
         assert oc == c and opk.tolist() == _packed(codes)
         assert Fraction(oe6) == e6 and Fraction(oe4) == e4
         chose4 += e4 < e6
+        subnormal_scales += 0 < (c & 0x7F) < 8  # e4m3 exponent field 0: a subnormal scale
         for R, rule in ((6, "static_6"), (4, "static_4")):
             sc, _, scodes = ex.candidate(bits, amax_t, R)
             occ, opk2, _, _ = orc.quantize_block_detail(x, amax_f, rule)
             assert occ == sc and opk2.tolist() == _packed(scodes)
     assert 0 < chose4 < len(blocks)
+    assert subnormal_scales > 10

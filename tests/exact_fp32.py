@@ -65,6 +65,23 @@ def rn32(q: Fraction) -> Fraction:
     return -r if neg else r
 
 
+def rn_bf16(q: Fraction) -> Fraction:
+    """Round an exact real to the nearest bf16 value (8 significant bits), ties to even
+    mantissa, subnormals included. Finite results only."""
+    if q == 0:
+        return Fraction(0)
+    a = abs(q)
+    e = max(_floor_log2(a), -126)
+    quantum = Fraction(2) ** (e - 7)
+    m = a / quantum
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    r = n * quantum
+    return -r if q < 0 else r
+
+
 def bf16_value(bits: int) -> Fraction:
     """Exact value of a bf16 bit pattern (finite)."""
     sign = -1 if bits & 0x8000 else 1

@@ -106,26 +106,6 @@ def test_rtn_relative_mse(orc, bits, bound):
 
 # ---------------------------------------------------------------- exact restatement
 
-def _rn_bf16(q):
-    """Round an exact real to the nearest bf16 value, ties to even (subnormals included)."""
-    from fractions import Fraction
-
-    import exact_fp32 as ex
-
-    if q == 0:
-        return Fraction(0)
-    a = abs(q)
-    e = max(ex._floor_log2(a), -126)
-    quantum = Fraction(2) ** (e - 7)
-    m = a / quantum
-    n = m.numerator // m.denominator
-    rem = m - n
-    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
-        n += 1
-    r = n * quantum
-    return -r if q < 0 else r
-
-
 def _round_half_even(t):
     from fractions import Fraction
 
@@ -155,10 +135,10 @@ def test_rtn_equals_exact_restatement(orc, bits):
         y = orc.rtn_dequantize(p, s, 16, bits)
         xs = [ex.bf16_value(int(b)) for b in x]
         amax_b = max(abs(t) for t in xs)
-        S = _rn_bf16(ex.rn32(amax_b / qmax))
+        S = ex.rn_bf16(ex.rn32(amax_b / qmax))
         assert ex.bf16_value(int(s[0])) == S, (trial, float(S))
         q = [0 if S == 0 else max(-qmax, min(qmax, _round_half_even(ex.rn32(t / S)))) for t in xs]
         assert _codes(p, bits).tolist() == q, trial
-        want = [_rn_bf16(ex.rn32(qi * S)) for qi in q]
+        want = [ex.rn_bf16(ex.rn32(qi * S)) for qi in q]
         assert [abs(ex.bf16_value(int(b))) for b in y] == [abs(w) for w in want], trial
         assert all(ex.bf16_value(int(b)) == w for b, w in zip(y, want) if w != 0), trial
